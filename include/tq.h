@@ -1,0 +1,227 @@
+/*
+ * tq.h -- C ABI of libtq, a B200 (sm_100a) library for TurboQuant-style
+ * online vector quantization: batched encode of fp32/bf16 vectors into packed
+ * low-bit codes plus a 1-bit QJL sketch of the residual, and asymmetric
+ * inner-product scoring of fp32 queries against those codes (all logits, or
+ * top-k).
+ *
+ * Sources of the method ("TurboQuant article" = the intelliparadigm.com page
+ * "TurboQuant 技术概览与核心价值"; "TurboQuant blog" = the blog.hotdry.top page
+ * "TurboQuant 深度解读"):
+ *   - online, training-free quantization ........ TurboQuant article 1.1, 3.3; blog 一
+ *   - random rotation (Haar, or 3 rounds of
+ *     +-1 diagonal then Walsh-Hadamard) .......... TurboQuant article 1.2.1, 2.1.1-2.1.2
+ *   - (b-1)-bit Lloyd-Max codebook on the
+ *     Beta((d-1)/2,(d-1)/2) coordinate law ....... TurboQuant article 1.2.2, 2.2.1-2.2.2
+ *   - residual + 1-bit QJL sketch, unbiased
+ *     inner products ............................. TurboQuant article 1.2.3, 2.3.1-2.3.2; blog 三
+ *   - stored L2 norm, same rotation on queries,
+ *     top-K retrieval ............................ TurboQuant article 4.2.1-4.2.2
+ *   - outlier channels at more bits (3.5-bit) ... TurboQuant article 3.2, 4.1.1; blog 四
+ *
+ * Conventions for every call:
+ *   - Return a tq_status; calls never abort and never throw across the ABI.
+ *     Arguments are validated before anything is launched; on error nothing
+ *     is written.  A CUDA launch error maps to TQ_ERR_CUDA; an asynchronous
+ *     fault surfaces at the next synchronization of the stream.
+ *   - Device calls are asynchronous on `stream` (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream) and run on the device that was
+ *     current when the quantizer was created.
+ *   - The caller allocates and frees every data buffer (device memory unless
+ *     stated).  The library owns only the quantizer's read-only device tables.
+ *   - A quantizer is immutable after creation and may be shared by threads.
+ *   - n == 0 (or nq == 0) is a successful no-op.
+ *
+ * Packed layouts (per vector, d a multiple of 32, m = d):
+ *   codes: w*d/8 bytes, w = b-1 bits per coordinate, in groups of 32
+ *          coordinates; group g occupies w 32-bit little-endian words
+ *          starting at word w*g.  Within a group (coordinate j = 32g + i):
+ *            w = 1: word 0 bit i                      = code
+ *            w = 2: word i/16, bits 4*(i%8) + 2*((i/8)%2) .. +1 = code
+ *            w = 3: i < 24: word i/8, bits 4*(i%8) .. +2 = code;
+ *                   i >= 24 (k = i-24): bit 4k+3 of words 0, 1, 2 hold
+ *                   code bits 2, 1, 0 respectively
+ *            w = 4: word i/8, bits 4*(i%8) .. +3 = code
+ *          (layouts chosen so that one logical AND / shift exposes 4-bit
+ *          byte selectors for the scorer's table lookups).
+ *   signs: m/8 bytes; bit i of 32-bit word i/32 is 1 iff (S r)_i >= 0.
+ *   norms: 2 floats: ||x|| and gamma = ||r||.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tq_quantizer tq_quantizer;
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad enum, ...        */
+  TQ_ERR_UNSUPPORTED = 2,  /* (d, b, m, rotation, dtype) outside what is built   */
+  TQ_ERR_ALIGNMENT = 3,    /* a pointer or leading dimension breaks the stated alignment */
+  TQ_ERR_NOMEM = 4,        /* host or device allocation of the quantizer tables failed */
+  TQ_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed        */
+  TQ_ERR_WORKSPACE = 6     /* workspace pointer null or smaller than required    */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+typedef enum {
+  TQ_ROT_AUTO = 0,      /* Hadamard for power-of-two d, Haar otherwise          */
+  TQ_ROT_HADAMARD = 1,  /* R = H D3 H D2 H D1 (orthonormal Walsh-Hadamard H)   */
+  TQ_ROT_HAAR = 2       /* seeded Haar orthogonal matrix, stored fp32          */
+} tq_rotation;
+
+typedef struct {
+  int d, b, w, m;          /* dimension, total bits, MSE bits (b-1), QJL rows */
+  int rotation;            /* TQ_ROT_HADAMARD or TQ_ROT_HAAR actually used     */
+  int device;              /* CUDA device the tables live on, -1 if host-only   */
+  uint64_t seed;
+  size_t code_bytes;       /* w*d/8  per vector */
+  size_t sign_bytes;       /* m/8    per vector */
+  double coord_mse;        /* Lloyd-Max distortion per coordinate, D_w          */
+} tq_info_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *tq_status_string(tq_status s);
+
+/* ---------------------------------------------------------------- set-up
+ * tq_codebook: build a quantizer on the current CUDA device.
+ *   d: dimension, a multiple of 32 in [32, 4096]; b: total bits per
+ *   coordinate in [2, 5] (w = b-1 MSE bits, then 1 QJL bit); m: QJL rows,
+ *   must equal d (0 = d); seed: selects every random draw; rot: rotation kind
+ *   (Hadamard needs power-of-two d).
+ * Host work: the w-bit Lloyd-Max quantizer of the coordinate density
+ * proportional to (1-x^2)^((d-3)/2) on [-1,1] (TurboQuant article 1.2.2,
+ * 2.2.1; fitted on the exact density, equal-probability start, symmetric,
+ * stops when no centroid moves by more than 1e-14 of the largest);
+ * D1..D3 in {+-1}^d or a Haar matrix (QR of a Gaussian matrix with the sign
+ * fix, TurboQuant article 1.2.1); S in R^{m x d} Gaussian stored at fp16
+ * precision (TurboQuant article 2.3.2).  Random draws use SplitMix64
+ * (Steele, Lea, Flood 2014) streams keyed by seed: stream 0-2 the diagonals,
+ * 3 the entries of S, 4 the Gaussian matrix of the Haar rotation;
+ * Box-Muller (cosine branch) turns word pairs into N(0,1).
+ * Deterministic in (d, b, m, seed, rot).  *out receives an owned handle;
+ * release it with tq_destroy. */
+tq_status tq_codebook(int d, int b, int m, uint64_t seed, tq_rotation rot,
+                      tq_quantizer **out);
+/* tq_codebook_host: the same tables, host memory only (no CUDA device is
+ * touched).  For inspection and cross-checks on machines without a GPU;
+ * device entry points return TQ_ERR_UNSUPPORTED for such a quantizer. */
+tq_status tq_codebook_host(int d, int b, int m, uint64_t seed, tq_rotation rot,
+                           tq_quantizer **out);
+void tq_destroy(tq_quantizer *q);
+tq_status tq_info(const tq_quantizer *q, tq_info_t *info);
+
+/* Host copies of the quantizer's tables, for inspection and cross-checks.
+ * centroids: 2^w doubles, thresholds: 2^w - 1 doubles (either may be NULL).
+ * rotation: d*d floats, row-major R (u = R x); Hadamard quantizers write the
+ * dense product H D3 H D2 H D1 rounded to fp32.  diag_signs: 3*d int8 (+-1,
+ * D1 then D2 then D3; Hadamard only, else untouched).  qjl: m*d fp16 bit
+ * patterns of S, row-major.  Any pointer may be NULL. */
+tq_status tq_codebook_get(const tq_quantizer *q, double *centroids,
+                          double *thresholds, double *coord_mse);
+tq_status tq_tables_get(const tq_quantizer *q, float *rotation,
+                        int8_t *diag_signs, uint16_t *qjl);
+
+/* ---------------------------------------------------------------- encode
+ * tq_encode: quantize n vectors (TurboQuant article 1.2.3, 2.3, 4.2.1).
+ *   x: device, row r at x + r*ldx elements of `dtype`; 16-byte aligned, and
+ *      ldx*sizeof(dtype) a multiple of 16.
+ *   chan: NULL, or device int32 [groups][d] channel map: coordinate j of row r
+ *      is x[r*ldx + chan[(r / chan_rows)*d + j]] (used to encode a subset of
+ *      channels, e.g. a head's outlier channels).  chan_rows > 0 when chan is
+ *      given.  Without chan, coordinate j is x[r*ldx + j] and ldx >= d.
+ *   codes, signs, norms: device outputs; row r is written at
+ *      codes + r*out_stride*code_bytes, signs + r*out_stride*sign_bytes,
+ *      norms + 2*r*out_stride (out_stride >= 1; a caller appends into a
+ *      cache by offsetting the pointers).  codes/signs 4-byte aligned, norms
+ *      8-byte aligned.
+ * Per row: ||x|| (fp32), x_hat = x/||x|| (0 for a zero row), u = R x_hat,
+ * code_j = #{thresholds < u_j}, r = u - c[code], gamma = ||r||,
+ * sign bit i = [(S r)_i >= 0]. */
+tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype,
+                    int64_t n, int64_t ldx, const int32_t *chan,
+                    int64_t chan_rows, void *codes, void *signs, float *norms,
+                    int64_t out_stride, void *stream);
+
+/* Scratch (bytes of device memory) tq_encode needs for n rows; 0 for
+ * Hadamard quantizers.  Haar quantizers process rows in batches through
+ * this workspace; pass it to tq_encode_ws. */
+size_t tq_encode_workspace_bytes(const tq_quantizer *q, int64_t n);
+tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype,
+                       int64_t n, int64_t ldx, const int32_t *chan,
+                       int64_t chan_rows, void *codes, void *signs,
+                       float *norms, int64_t out_stride, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------- queries
+ * tq_prepare_queries: y~ = R y and p = S y~ in fp32 (the same rotation as the
+ * keys, TurboQuant article 4.2.2).  y: device fp32, row i at y + i*ldy (or
+ * gathered through ychan [groups][d] with group = i / ychan_rows, as in
+ * tq_encode).  ytil: nq x d, p: nq x m, device fp32, caller-allocated. */
+tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq,
+                             int64_t ldy, const int32_t *ychan,
+                             int64_t ychan_rows, float *ytil, float *p,
+                             void *stream);
+
+/* ---------------------------------------------------------------- score
+ * tq_score: asymmetric estimate of <y, x> for grouped keys and queries
+ * (KV-cache attention logits; blog 四).
+ *   Keys: groups*keys_per_group encoded rows (codes/signs/norms as written by
+ *   tq_encode with out_stride 1); key k of group g is row g*keys_per_group+k.
+ *   Queries: groups*G fp32 rows of y (ldy, optional ychan gather with
+ *   ychan_rows = G); query i of group g is row g*G + i.
+ *   out: device fp32 [groups*G][keys_per_group]; query row g*G+i, column k
+ *   receives s = ||x|| * (<y~, c[codes]> + gamma*sqrt(pi/2)/m * <p, 2*bits-1>)
+ *   (added to the existing value when accumulate != 0).
+ *   workspace: device, at least tq_score_workspace_bytes(q, groups*G) bytes,
+ *   16-byte aligned (holds the prepared queries). */
+size_t tq_score_workspace_bytes(const tq_quantizer *q, int64_t nq);
+tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups,
+                   int64_t G, int64_t ldy, const int32_t *ychan,
+                   const void *codes, const void *signs, const float *norms,
+                   int64_t keys_per_group, float *out, int accumulate,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------- top-k
+ * tq_topk: the k highest estimates per query over n keys (TurboQuant article
+ * 4.2.2, first stage of two-stage retrieval).  y: nq fp32 rows (ldy).
+ * out_scores: nq x k fp32, out_idx: nq x k int64 (device), sorted by
+ * descending score, equal scores by ascending key index.  1 <= k <= 64 and
+ * k <= n.  workspace: at least tq_topk_workspace_bytes(q, nq, n, k) bytes. */
+size_t tq_topk_workspace_bytes(const tq_quantizer *q, int64_t nq, int64_t n,
+                               int k);
+tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq,
+                  int64_t ldy, const void *codes, const void *signs,
+                  const float *norms, int64_t n, int k, float *out_scores,
+                  int64_t *out_idx, void *workspace, size_t workspace_bytes,
+                  void *stream);
+
+/* ---------------------------------------------------------------- outliers
+ * tq_outlier_channels: per group of rows, the `count` channels of highest
+ * mean square (the outlier channels kept at more bits; TurboQuant article
+ * 4.1.1 suggests about 25%).  x: device, groups*rows_per_group rows of `dim`
+ * channels (ldx, dtype).  Sums of squares are accumulated in fp64 on the
+ * device; ties go to the lower channel index.  out_sel: device int32
+ * [groups][count] selected channels ascending; out_rest: device int32
+ * [groups][dim-count] the other channels ascending (either may be NULL).
+ * workspace: tq_outlier_workspace_bytes(groups, dim) bytes.  Synchronizes
+ * `stream` (the selection runs on the host). */
+size_t tq_outlier_workspace_bytes(int64_t groups, int dim);
+tq_status tq_outlier_channels(const void *x, tq_dtype dtype, int64_t groups,
+                              int64_t rows_per_group, int dim, int64_t ldx,
+                              int count, int32_t *out_sel, int32_t *out_rest,
+                              void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

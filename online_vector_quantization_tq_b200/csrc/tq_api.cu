@@ -1,0 +1,267 @@
+// C ABI entry points of libtq that launch device work (encode, query
+// preparation, scoring, top-k, outlier-channel choice).  Argument checks
+// happen here, before anything is launched; see include/tq.h for the
+// contract of each call.
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "tq_kernels.h"
+
+namespace {
+
+using namespace tq;
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      ok = false;
+      return;
+    }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline bool fwht_fast(const tq_quantizer *q) {
+  return q->rotation == TQ_ROT_HADAMARD && (q->d == 32 || q->d == 64 || q->d == 128);
+}
+
+tq_status check_rows(const tq_quantizer *q, const void *x, int dtype, int64_t n, int64_t ldx,
+                     const int32_t *chan, int64_t chan_rows) {
+  if (!q || !x || n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_ERR_INVALID_ARG;
+  if (q->device < 0) return TQ_ERR_UNSUPPORTED;  // host-only quantizer
+  if (chan ? chan_rows <= 0 : ldx < q->d) return TQ_ERR_INVALID_ARG;
+  if (ldx < 1) return TQ_ERR_INVALID_ARG;
+  const size_t es = dtype == TQ_BF16 ? 2 : 4;
+  if (!aligned(x, 16) || ((size_t)ldx * es) % 16 != 0) return TQ_ERR_ALIGNMENT;
+  if (chan && !aligned(chan, 4)) return TQ_ERR_ALIGNMENT;
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t tq_encode_workspace_bytes(const tq_quantizer *q, int64_t n) {
+  if (!q || n <= 0 || fwht_fast(q)) return 0;
+  return round_up(v1_dense_ws_bytes(q, n), 256);
+}
+
+tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_t n, int64_t ldx,
+                       const int32_t *chan, int64_t chan_rows, void *codes, void *signs, float *norms,
+                       int64_t out_stride, void *workspace, size_t workspace_bytes, void *stream) {
+  tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows);
+  if (st != TQ_OK) return st;
+  if (!codes || !signs || !norms || out_stride < 1) return TQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8)) return TQ_ERR_ALIGNMENT;
+  if (n == 0) return TQ_OK;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RowSource src{x, ldx, chan, chan_rows, q->d, dtype == TQ_BF16};
+  if (fwht_fast(q)) return v1_encode_fwht(q, src, n, codes, signs, norms, out_stride, s);
+  if (!workspace || !aligned(workspace, 16) || v1_dense_batch_rows(q, workspace_bytes) < 1)
+    return TQ_ERR_WORKSPACE;
+  return v1_encode_dense(q, src, n, codes, signs, norms, out_stride, workspace, workspace_bytes, s);
+}
+
+tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_t n, int64_t ldx,
+                    const int32_t *chan, int64_t chan_rows, void *codes, void *signs, float *norms,
+                    int64_t out_stride, void *stream) {
+  if (!q) return TQ_ERR_INVALID_ARG;
+  const size_t ws = tq_encode_workspace_bytes(q, n);
+  if (ws == 0)
+    return tq_encode_ws(q, x, dtype, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, nullptr, 0,
+                        stream);
+  tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows);
+  if (st != TQ_OK) return st;
+  if (!codes || !signs || !norms || out_stride < 1) return TQ_ERR_INVALID_ARG;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void *buf = nullptr;
+  if (cudaMallocAsync(&buf, ws, s) != cudaSuccess) {
+    cudaGetLastError();
+    return TQ_ERR_NOMEM;
+  }
+  st = tq_encode_ws(q, x, dtype, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, buf, ws, stream);
+  cudaFreeAsync(buf, s);
+  return st;
+}
+
+tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy,
+                             const int32_t *ychan, int64_t ychan_rows, float *ytil, float *p, void *stream) {
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, ychan_rows);
+  if (st != TQ_OK) return st;
+  if (!ytil || !p) return TQ_ERR_INVALID_ARG;
+  if (!aligned(ytil, 16) || !aligned(p, 16)) return TQ_ERR_ALIGNMENT;
+  if (nq == 0) return TQ_OK;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  RowSource src{y, ldy, ychan, ychan_rows, q->d, 0};
+  return v1_prepare_queries(q, src, nq, ytil, p, static_cast<cudaStream_t>(stream));
+}
+
+size_t tq_score_workspace_bytes(const tq_quantizer *q, int64_t nq) {
+  if (!q || nq <= 0) return 0;
+  return round_up((size_t)nq * q->d * 4, 256) + round_up((size_t)nq * q->m * 4, 256);
+}
+
+tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_t G, int64_t ldy,
+                   const int32_t *ychan, const void *codes, const void *signs, const float *norms,
+                   int64_t keys_per_group, float *out, int accumulate, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+  if (!q || groups < 0 || G < 0 || keys_per_group < 0) return TQ_ERR_INVALID_ARG;
+  const int64_t nq = groups * G;
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, G > 0 ? G : 1);
+  if (st != TQ_OK) return st;
+  if (!codes || !signs || !norms || !out) return TQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out, 4)) return TQ_ERR_ALIGNMENT;
+  if (nq == 0 || keys_per_group == 0) return TQ_OK;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < tq_score_workspace_bytes(q, nq))
+    return TQ_ERR_WORKSPACE;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *ytil = static_cast<float *>(workspace);
+  float *p = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up((size_t)nq * q->d * 4, 256));
+  RowSource src{y, ldy, ychan, G, q->d, 0};
+  st = v1_prepare_queries(q, src, nq, ytil, p, s);
+  if (st != TQ_OK) return st;
+  return v1_score(q, ytil, p, nq, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
+                  keys_per_group, accumulate, s);
+}
+
+}  // extern "C"
+
+namespace {
+constexpr int64_t kTopkChunk = 65536;
+constexpr int64_t kTopkSlice = 2048;
+
+struct TopkLayout {
+  size_t ytil, p, scores, part_s, part_i, total;
+  int64_t chunk, nparts;
+};
+
+TopkLayout topk_layout(const tq_quantizer *q, int64_t nq, int64_t n, int k) {
+  TopkLayout L{};
+  L.chunk = std::min<int64_t>(n, kTopkChunk);
+  L.nparts = (n + kTopkSlice - 1) / kTopkSlice;
+  size_t off = 0;
+  L.ytil = off;
+  off += round_up((size_t)nq * q->d * 4, 256);
+  L.p = off;
+  off += round_up((size_t)nq * q->m * 4, 256);
+  L.scores = off;
+  off += round_up((size_t)nq * L.chunk * 4, 256);
+  L.part_s = off;
+  off += round_up((size_t)nq * L.nparts * k * 4, 256);
+  L.part_i = off;
+  off += round_up((size_t)nq * L.nparts * k * 8, 256);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+extern "C" {
+
+size_t tq_topk_workspace_bytes(const tq_quantizer *q, int64_t nq, int64_t n, int k) {
+  if (!q || nq <= 0 || n <= 0 || k <= 0) return 0;
+  return topk_layout(q, nq, n, k).total;
+}
+
+tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy, const void *codes,
+                  const void *signs, const float *norms, int64_t n, int k, float *out_scores, int64_t *out_idx,
+                  void *workspace, size_t workspace_bytes, void *stream) {
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, nullptr, 0);
+  if (st != TQ_OK) return st;
+  if (n < 0 || !codes || !signs || !norms || !out_scores || !out_idx) return TQ_ERR_INVALID_ARG;
+  if (nq == 0) return TQ_OK;
+  if (k < 1 || k > 64 || k > n) return TQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out_idx, 8) ||
+      !aligned(out_scores, 4))
+    return TQ_ERR_ALIGNMENT;
+  const TopkLayout L = topk_layout(q, nq, n, k);
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < L.total) return TQ_ERR_WORKSPACE;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  float *ytil = reinterpret_cast<float *>(ws + L.ytil);
+  float *p = reinterpret_cast<float *>(ws + L.p);
+  float *scores = reinterpret_cast<float *>(ws + L.scores);
+  float *part_s = reinterpret_cast<float *>(ws + L.part_s);
+  int64_t *part_i = reinterpret_cast<int64_t *>(ws + L.part_i);
+  RowSource src{y, ldy, nullptr, 0, q->d, 0};
+  st = v1_prepare_queries(q, src, nq, ytil, p, s);
+  if (st != TQ_OK) return st;
+  for (int64_t c0 = 0; c0 < n; c0 += L.chunk) {
+    const int64_t cnt = std::min(L.chunk, n - c0);
+    st = v1_score(q, ytil, p, nq, nq, n, c0, cnt, codes, signs, norms, scores, L.chunk, 0, s);
+    if (st != TQ_OK) return st;
+    st = v1_topk_select(scores, nullptr, nq, L.chunk, cnt, kTopkSlice, c0, k, part_s + (c0 / kTopkSlice) * k,
+                        part_i + (c0 / kTopkSlice) * k, L.nparts * k, s);
+    if (st != TQ_OK) return st;
+  }
+  return v1_topk_select(part_s, part_i, nq, L.nparts * k, L.nparts * k, L.nparts * k, 0, k, out_scores, out_idx,
+                        k, s);
+}
+
+size_t tq_outlier_workspace_bytes(int64_t groups, int dim) {
+  if (groups <= 0 || dim <= 0) return 0;
+  return round_up((size_t)groups * 64 * dim * 8, 256) + round_up((size_t)groups * dim * 8, 256);
+}
+
+tq_status tq_outlier_channels(const void *x, tq_dtype dtype, int64_t groups, int64_t rows_per_group, int dim,
+                              int64_t ldx, int count, int32_t *out_sel, int32_t *out_rest, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+  if (!x || groups < 0 || rows_per_group < 0 || dim <= 0 || ldx < dim || count < 0 || count > dim ||
+      (dtype != TQ_F32 && dtype != TQ_BF16))
+    return TQ_ERR_INVALID_ARG;
+  const size_t es = dtype == TQ_BF16 ? 2 : 4;
+  if (!aligned(x, 16) || ((size_t)ldx * es) % 16 != 0) return TQ_ERR_ALIGNMENT;
+  if (groups == 0) return TQ_OK;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < tq_outlier_workspace_bytes(groups, dim))
+    return TQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double *part = static_cast<double *>(workspace);
+  double *fin = reinterpret_cast<double *>(static_cast<char *>(workspace) + round_up((size_t)groups * 64 * dim * 8, 256));
+  const int nchunks = (int)std::max<int64_t>(1, std::min<int64_t>(64, rows_per_group));
+  RowSource src{x, ldx, nullptr, 0, dim, dtype == TQ_BF16};
+  tq_status st = v1_sumsq(src, groups, rows_per_group, part, nchunks, fin, s);
+  if (st != TQ_OK) return st;
+  std::vector<double> ms((size_t)groups * dim);
+  if (cudaMemcpyAsync(ms.data(), fin, ms.size() * 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  std::vector<int32_t> sel((size_t)groups * count), rest((size_t)groups * (dim - count));
+  std::vector<int> order(dim);
+  for (int64_t gi = 0; gi < groups; ++gi) {
+    const double *v = &ms[(size_t)gi * dim];
+    for (int c = 0; c < dim; ++c) order[c] = c;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return v[a] > v[b]; });
+    std::vector<int> a(order.begin(), order.begin() + count), b(order.begin() + count, order.end());
+    std::sort(a.begin(), a.end());
+    std::sort(b.begin(), b.end());
+    std::copy(a.begin(), a.end(), sel.begin() + gi * count);
+    std::copy(b.begin(), b.end(), rest.begin() + gi * (dim - count));
+  }
+  if (out_sel && count > 0 &&
+      cudaMemcpyAsync(out_sel, sel.data(), sel.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (out_rest && dim - count > 0 &&
+      cudaMemcpyAsync(out_rest, rest.data(), rest.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// Internal definitions shared by the host set-up code and the CUDA kernels
+// of libtq.  Not part of the public ABI (see include/tq.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr int kMaxLevels = 16;  // 2^w for w <= 4
+
+// Small, POD view of a quantizer that kernels take by value.
+struct KernelTables {
+  int d, w, m, levels;
+  float centroids[kMaxLevels];
+  float thresholds[kMaxLevels];       // levels-1 used; rest +inf
+  float qjl_scale;                    // sqrt(pi/2) / m
+  const uint32_t *diag_bits;          // Hadamard: 3 x d/32 words, bit set = -1
+  const float *rot;                   // Haar: d x d row-major fp32 (u = R x)
+  const uint16_t *qjl16;              // m x d fp16 bit patterns of S
+  const float *qjl32;                 // m x d fp32 values of S (same numbers)
+};
+
+}  // namespace tq
+
+struct tq_quantizer {
+  int d = 0, b = 0, w = 0, m = 0, rotation = 0, device = 0;
+  uint64_t seed = 0;
+  std::vector<double> centroids, thresholds;
+  double coord_mse = 0.0;
+  std::vector<float> rot;        // d x d fp32 (Haar, or the dense Hadamard product)
+  std::vector<int8_t> diag;      // 3 x d (Hadamard)
+  std::vector<uint16_t> qjl16;   // m x d fp16 bits
+  // device copies (owned)
+  uint32_t *d_diag_bits = nullptr;
+  float *d_rot = nullptr;
+  uint16_t *d_qjl16 = nullptr;
+  float *d_qjl32 = nullptr;
+  tq::KernelTables kt{};
+};
+
+namespace tq {
+// Host-side helpers exported for the CUDA translation unit.
+uint16_t double_to_half_bits(double v);
+double half_bits_to_double(uint16_t h);
+}  // namespace tq

@@ -1,0 +1,29 @@
+// Internal kernel entry points of libtq (called by the C ABI in tq_api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "tq_common.cuh"
+
+namespace tq {
+
+tq_status v1_encode_fwht(const tq_quantizer *q, const RowSource &src, int64_t n, void *codes,
+                         void *signs, float *norms, int64_t out_stride, cudaStream_t st);
+size_t v1_dense_ws_bytes(const tq_quantizer *q, int64_t n);
+size_t v1_dense_batch_rows(const tq_quantizer *q, size_t ws_bytes);
+tq_status v1_encode_dense(const tq_quantizer *q, const RowSource &src, int64_t n, void *codes,
+                          void *signs, float *norms, int64_t out_stride, void *ws, size_t ws_bytes,
+                          cudaStream_t st);
+tq_status v1_prepare_queries(const tq_quantizer *q, const RowSource &src, int64_t nq, float *ytil,
+                             float *p, cudaStream_t st);
+tq_status v1_score(const tq_quantizer *q, const float *ytil, const float *p, int64_t nq_rows, int64_t G,
+                   int64_t keys_per_group, int64_t key_base, int64_t nkeys, const void *codes,
+                   const void *signs, const float *norms, float *out, int64_t ldo, int accumulate,
+                   cudaStream_t st);
+tq_status v1_topk_select(float *score, const int64_t *idx, int64_t rows, int64_t row_stride, int64_t cnt,
+                         int64_t slice, int64_t base, int k, float *out_s, int64_t *out_i,
+                         int64_t out_row_stride, cudaStream_t st);
+tq_status v1_sumsq(const RowSource &src, int64_t groups, int64_t rows_per_group, double *part, int nchunks,
+                   double *out, cudaStream_t st);
+
+}  // namespace tq

@@ -1,0 +1,264 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the fp64
+oracle on the same seeded inputs, for the five workloads and the edge cases.
+Rules (exemptions, tolerances) are in tests/parity.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import tq_oracle as o
+from tests.parity import check_encode, check_scores, check_topk, score_errors
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tq():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from online_vector_quantization_tq_b200 import build
+    build.build()
+    import online_vector_quantization_tq_b200 as pkg
+    pkg.lib()
+    return pkg
+
+
+_TABLES = {}
+
+
+def tables(d, b, rot="auto"):
+    key = (d, b, rot)
+    if key not in _TABLES:
+        _TABLES[key] = o.Tables(d, b, seed=wl.QUANTIZER_SEED, rotation=rot)
+    return _TABLES[key]
+
+
+def host(enc, rows=None):
+    sl = slice(None) if rows is None else rows
+    return (enc.codes[sl].cpu().numpy(), enc.signs[sl].cpu().numpy(), enc.norms[sl].cpu().numpy())
+
+
+def dev(a, dtype=torch.float32):
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda").to(dtype)
+
+
+# ------------------------------------------------------------------ tiny
+
+def test_tiny_encode_score_topk(tq):
+    x = wl.tiny_keys()
+    y = wl.tiny_queries()
+    t = tables(128, 3)
+    q = tq.tq_codebook(128, 3, seed=wl.QUANTIZER_SEED)
+    enc = tq.tq_encode(q, dev(x))
+    rep = check_encode(*host(enc), x, t)
+    ytil, p = o.prepare_query(y, t)
+    s_ref = o.score(ytil, p, rep.ref, t)
+    s = tq.tq_score(q, dev(y), 1, 16, enc, 4096).cpu().numpy()
+    check_scores(s, s_ref, rep.ref["norm"], np.linalg.norm(y, axis=1), 128, rep.skip_rows)
+    vals, idx = tq.tq_topk(q, dev(y), enc, 10)
+    vals, idx = vals.cpu().numpy(), idx.cpu().numpy()
+    check_topk(vals, idx, s_ref, rep.ref["norm"], np.linalg.norm(y, axis=1), 128, 10)
+    # top-k scores are the scorer's own values, bit for bit
+    assert np.array_equal(vals, np.take_along_axis(s, idx, axis=1))
+
+
+def test_prepared_queries(tq):
+    y = wl.tiny_queries()
+    for d, b in ((128, 3), (96, 3), (32, 5)):
+        t = tables(d, b)
+        q = tq.tq_codebook(d, b, seed=0)
+        yy = y[:, :d].copy()
+        ytil, p = tq.tq_prepare_queries(q, dev(yy))
+        rt, rp = o.prepare_query(yy, t)
+        assert np.allclose(ytil.cpu().numpy(), rt, rtol=0, atol=2e-5 * np.abs(rt).max())
+        assert np.allclose(p.cpu().numpy(), rp, rtol=0, atol=2e-5 * np.abs(rp).max())
+
+
+# ------------------------------------------------------------------ kv (8B-class GQA layer)
+
+def _kv_tensor(n=131072):
+    return np.stack([wl.kv_head_keys(h, n) for h in range(8)])  # [8, n, 128] bf16-exact fp32
+
+
+def test_kv_full(tq):
+    n = 131072
+    xs = _kv_tensor(n)
+    y = wl.kv_queries()
+    t = tables(128, 4)
+    q = tq.tq_codebook(128, 4, seed=0)
+    x_dev = dev(xs.reshape(-1, 128), torch.bfloat16)
+    enc = tq.tq_encode(q, x_dev)
+    out = tq.tq_score(q, dev(y), 8, 4, enc, n).cpu().numpy()
+    worst, exempt = 0.0, 0
+    for h in range(8):
+        rows = slice(h * n, (h + 1) * n)
+        rep = check_encode(*host(enc, rows), xs[h], t)
+        exempt += rep.n_code_exempt + rep.n_sign_exempt
+        yh = y[4 * h:4 * h + 4]
+        s_ref = o.score(*o.prepare_query(yh, t), rep.ref, t)
+        worst = max(worst, check_scores(out[4 * h:4 * h + 4], s_ref, rep.ref["norm"],
+                                        np.linalg.norm(yh, axis=1), 128, rep.skip_rows))
+    print(f"kv: exempt coordinates {exempt}, worst score error {worst:.2e}")
+
+
+# ------------------------------------------------------------------ kv_mixed (3.5-bit split)
+
+def test_kv_mixed_full(tq):
+    n = 131072
+    xs = _kv_tensor(n)
+    y = wl.kv_queries()
+    x_dev = dev(xs.reshape(-1, 128), torch.bfloat16)
+    sel, rest = tq.tq_outlier_channels(x_dev, 8, n, 32)
+    sel, rest = sel.cpu().numpy(), rest.cpu().numpy()
+    for h in range(8):
+        ref_sel = o.outlier_channels(xs[h], 32)
+        assert np.array_equal(sel[h], ref_sel)
+        assert np.array_equal(rest[h], np.setdiff1d(np.arange(128), ref_sel))
+        assert set(wl.kv_outlier_channels(h)) <= set(ref_sel.tolist())
+    (da, ba), (db, bb) = wl.MIXED_SPLIT
+    qa, qb = tq.tq_codebook(da, ba, seed=0), tq.tq_codebook(db, bb, seed=0)
+    ta, tb = tables(da, ba), tables(db, bb)
+    sel_d, rest_d = dev(sel, torch.int32), dev(rest, torch.int32)
+    ea = tq.tq_encode(qa, x_dev, chan=sel_d, chan_rows=n)
+    eb = tq.tq_encode(qb, x_dev, chan=rest_d, chan_rows=n)
+    y_dev = dev(y)
+    out = tq.tq_score(qa, y_dev, 8, 4, ea, n, ychan=sel_d)
+    tq.tq_score(qb, y_dev, 8, 4, eb, n, out=out, accumulate=True, ychan=rest_d)
+    out = out.cpu().numpy()
+    worst = 0.0
+    for h in range(8):
+        rows = slice(h * n, (h + 1) * n)
+        ra = check_encode(*host(ea, rows), xs[h][:, sel[h]], ta)
+        rb = check_encode(*host(eb, rows), xs[h][:, rest[h]], tb)
+        yh = y[4 * h:4 * h + 4]
+        s_ref = (o.score(*o.prepare_query(yh[:, sel[h]], ta), ra.ref, ta)
+                 + o.score(*o.prepare_query(yh[:, rest[h]], tb), rb.ref, tb))
+        worst = max(worst, check_scores(out[4 * h:4 * h + 4], s_ref, np.linalg.norm(xs[h], axis=1),
+                                        np.linalg.norm(yh, axis=1), 128, ra.skip_rows | rb.skip_rows))
+    print(f"kv_mixed: worst score error {worst:.2e}")
+
+
+# ------------------------------------------------------------------ decode step
+
+def test_decode_step_full_size(tq):
+    groups, n = 256, 32768
+    t = tables(128, 3)
+    q = tq.tq_codebook(128, 3, seed=0)
+    x = torch.empty((groups * n, 128), dtype=torch.bfloat16, device="cuda")
+    for g in range(groups):
+        x[g * n:(g + 1) * n] = dev(wl.decode_group_keys(g, n), torch.bfloat16)
+    cache = q.empty_encoded(groups * n)
+    # the cache: the first n-1 keys of every group, written group by group
+    for g in range(groups):
+        part = tq.binding.Encoded(cache.codes[g * n:], cache.signs[g * n:], cache.norms[g * n:])
+        tq.tq_encode(q, x[g * n:g * n + n - 1], out=part)
+    # the decode step: one new key per group appended in place (out_stride = n)
+    new = x.view(groups, n, 128)[:, n - 1, :].contiguous()
+    tail = tq.binding.Encoded(cache.codes[n - 1:], cache.signs[n - 1:], cache.norms[n - 1:])
+    tq.tq_encode(q, new, out=tail, out_stride=n)
+    y = wl.decode_queries(groups)
+    out = tq.tq_score(q, dev(y), groups, 4, cache, n).cpu().numpy()
+    for g in (0, 131, 255):
+        xg = wl.decode_group_keys(g, n)
+        rows = slice(g * n, (g + 1) * n)
+        rep = check_encode(*host(cache, rows), xg, t)
+        yg = y[4 * g:4 * g + 4]
+        s_ref = o.score(*o.prepare_query(yg, t), rep.ref, t)
+        check_scores(out[4 * g:4 * g + 4], s_ref, rep.ref["norm"], np.linalg.norm(yg, axis=1), 128,
+                     rep.skip_rows)
+
+
+# ------------------------------------------------------------------ ANN d=1536
+
+def test_ann_full_size_sampled(tq):
+    n, d, nq = 1_000_000, 1536, 16
+    t = tables(d, 4)
+    q = tq.tq_codebook(d, 4, seed=0)
+    x = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    for c in range((n + wl.ANN_CHUNK - 1) // wl.ANN_CHUNK):
+        blk = wl.ann_chunk(c, n, d)
+        x[c * wl.ANN_CHUNK:c * wl.ANN_CHUNK + blk.shape[0]] = dev(blk)
+    enc = tq.tq_encode(q, x)
+    rng = np.random.default_rng(7)
+    rows = np.unique(np.concatenate([np.arange(64), n - 64 + np.arange(64), rng.integers(0, n, 1024)]))
+    xr = wl.ann_rows(rows, n, d)
+    rep = check_encode(enc.codes[rows].cpu().numpy(), enc.signs[rows].cpu().numpy(),
+                       enc.norms[rows].cpu().numpy(), xr, t)
+    y = wl.ann_queries(1024, d)[:nq]
+    y_dev = dev(y)
+    s_all = tq.tq_score(q, y_dev, 1, nq, enc, n)
+    s_ref = o.score(*o.prepare_query(y, t), rep.ref, t)
+    check_scores(s_all[:, rows].cpu().numpy(), s_ref, rep.ref["norm"], np.linalg.norm(y, axis=1), d,
+                 rep.skip_rows)
+    vals, idx = tq.tq_topk(q, y_dev, enc, 10)
+    # top-k equals the top-k of the full score rows (same kernel arithmetic)
+    sv, si = torch.sort(s_all, dim=1, descending=True, stable=True)
+    assert torch.equal(vals, sv[:, :10]) and torch.equal(idx, si[:, :10])
+    # returned keys re-scored by the oracle
+    got = idx.cpu().numpy()
+    for qi in range(4):
+        xr2 = wl.ann_rows(got[qi], n, d)
+        r2 = o.encode(xr2, t)
+        ref_s = o.score(*o.prepare_query(y[qi:qi + 1], t), r2, t)
+        check_scores(vals[qi:qi + 1].cpu().numpy(), ref_s, r2["norm"], np.linalg.norm(y[qi:qi + 1], axis=1), d)
+    exact = y_dev @ x.T
+    truth = torch.topk(exact, 10, dim=1).indices.cpu().numpy()
+    recall = np.mean([len(set(got[i]) & set(truth[i])) / 10 for i in range(nq)])
+    print(f"ann recall@10 = {recall:.3f}")
+    assert recall >= 0.5
+
+
+# ------------------------------------------------------------------ dense paths and edge cases
+
+@pytest.mark.parametrize("d,b,rot", [(128, 4, "haar"), (256, 3, "hadamard"), (64, 2, "auto"), (32, 5, "auto")])
+def test_other_shapes(tq, d, b, rot):
+    rng = np.random.default_rng(d + b)
+    x = rng.standard_normal((1000, d)).astype(np.float32)
+    y = rng.standard_normal((5, d)).astype(np.float32)
+    t = tables(d, b, rot)
+    q = tq.tq_codebook(d, b, seed=0, rotation=rot)
+    enc = tq.tq_encode(q, dev(x))
+    rep = check_encode(*host(enc), x, t)
+    s = tq.tq_score(q, dev(y), 1, 5, enc, 1000).cpu().numpy()
+    check_scores(s, o.score(*o.prepare_query(y, t), rep.ref, t), rep.ref["norm"], np.linalg.norm(y, axis=1),
+                 d, rep.skip_rows)
+
+
+def test_edge_cases(tq):
+    t = tables(128, 3)
+    q = tq.tq_codebook(128, 3, seed=0)
+    rng = np.random.default_rng(3)
+    # ragged n, a zero row, bf16 with padded leading dimension
+    x = rng.standard_normal((333, 128)).astype(np.float32)
+    x[5] = 0.0
+    xb = wl.to_bf16_values(x)
+    pad = torch.zeros((333, 136), dtype=torch.bfloat16, device="cuda")
+    pad[:, :128] = dev(xb, torch.bfloat16)
+    enc = tq.tq_encode(q, pad[:, :128])
+    rep = check_encode(*host(enc), xb, t)
+    assert enc.norms[5, 0].item() == 0.0
+    s = tq.tq_score(q, dev(xb[:3]), 1, 3, enc, 333).cpu().numpy()
+    assert np.all(s[:, 5] == 0.0)
+    # n = 1 and n = 0
+    one = tq.tq_encode(q, dev(x[:1]))
+    check_encode(*host(one), x[:1], t)
+    empty = q.empty_encoded(0)
+    tq.tq_encode(q, torch.empty((0, 128), device="cuda"), out=empty)
+    # channel gather: a permutation of 160 input channels
+    wide = rng.standard_normal((200, 160)).astype(np.float32)
+    perm = rng.permutation(160)[:128].astype(np.int32)
+    enc2 = tq.tq_encode(q, dev(wide), chan=dev(perm[None, :], torch.int32), chan_rows=200)
+    check_encode(*host(enc2), wide[:, perm], t)
+    # argument errors return a status and launch nothing
+    xx = dev(x)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_encode(q, xx.view(-1)[1:].view(-1)[:128 * 100].view(100, 128))
+    assert e.value.code == 3
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_score(q, xx[:2], 1, 2, enc, 333, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == 6
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_topk(q, xx[:2], enc, 65)
+    assert e.value.code == 1
+    torch.cuda.synchronize()

@@ -1,0 +1,102 @@
+"""CPU-only checks of libtq: it loads, exports every entry point of
+include/tq.h, validates arguments, and its host-built tables (codebook,
+rotation, QJL projection) agree with the oracle's independent construction."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import tq_oracle as o
+from tests.layout import code_bit_position
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from online_vector_quantization_tq_b200 import build
+    build.build()
+    import online_vector_quantization_tq_b200 as pkg
+    pkg.lib()
+    return pkg
+
+
+def test_exports_every_declared_symbol(tq):
+    hdr = open(os.path.join(ROOT, "include", "tq.h")).read()
+    names = set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", hdr))
+    assert len(names) >= 15
+    so = ctypes.CDLL(tq.binding.LIB_PATH)
+    for name in sorted(names):
+        assert hasattr(so, name), name
+
+
+def test_status_strings(tq):
+    L = tq.lib()
+    for code in range(7):
+        assert L.tq_status_string(code)
+    assert L.tq_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("d,b,rot", [(128, 3, "auto"), (128, 4, "auto"), (32, 5, "auto"), (64, 2, "auto"),
+                                     (96, 3, "auto"), (256, 3, "haar"), (1536, 4, "auto")])
+def test_host_tables_match_oracle(tq, d, b, rot):
+    q = tq.tq_codebook_host(d, b, seed=0, rotation=rot)
+    t = o.Tables(d, b, seed=0, rotation=rot)
+    c, thr, mse = q.codebook()
+    scale = np.max(np.abs(t.centroids))
+    assert np.max(np.abs(c - t.centroids)) < 1e-12 * scale
+    assert np.max(np.abs(thr - t.thresholds)) < 1e-12 * scale
+    assert abs(mse - t.coord_mse) < 1e-12 * mse
+    R, diag, S = q.tables()
+    assert np.array_equal(S.view(np.float16).astype(np.float64), t.S)
+    if q.rotation == "hadamard":
+        for r, stream in enumerate((o.STREAM_D1, o.STREAM_D2, o.STREAM_D3)):
+            assert np.array_equal(diag[r].astype(np.float64), o.rademacher(0, stream, d))
+        # the dense product rounded once to fp32
+        assert np.all(np.abs(R.astype(np.float64) - t.R) <= np.abs(t.R) * 2.0 ** -24 + 1e-15)
+    else:
+        # same fp32 matrix up to rare one-ulp differences from the two QR codes
+        diff = R.astype(np.float64) - t.R
+        assert np.max(np.abs(diff)) <= np.max(np.abs(t.R)) * 2.0 ** -23
+        assert np.count_nonzero(diff) <= max(4, d * d // 100000)
+
+
+def test_deterministic_in_seed(tq):
+    a = tq.tq_codebook_host(128, 3, seed=7).tables()
+    b = tq.tq_codebook_host(128, 3, seed=7).tables()
+    c = tq.tq_codebook_host(128, 3, seed=8).tables()
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    assert not np.array_equal(a[2], c[2])
+
+
+@pytest.mark.parametrize("args,code", [((100, 3), 2), ((128, 1), 1), ((128, 6), 1), ((0, 3), 1),
+                                       ((4128, 3), 2)])
+def test_codebook_argument_errors(tq, args, code):
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_codebook_host(*args)
+    assert e.value.code == code
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_codebook_host(96, 3, rotation="hadamard")
+    assert e.value.code == 2
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_codebook_host(64, 3, m=32)
+    assert e.value.code == 2
+
+
+def test_device_calls_refuse_host_only_quantizer(tq):
+    """No GPU needed: the check happens before any pointer is touched."""
+    q = tq.tq_codebook_host(128, 3)
+    L = tq.lib()
+    fake = ctypes.c_void_p(0x1000)
+    st = L.tq_encode(q.handle, fake, 0, 16, 128, None, 0, fake, fake, fake, 1, None)
+    assert st == 2
+    st = L.tq_encode(None, fake, 0, 16, 128, None, 0, fake, fake, fake, 1, None)
+    assert st == 1
+
+
+def test_layout_is_a_bijection():
+    for w in (1, 2, 3, 4):
+        pos = sorted(code_bit_position(w, i, b) for i in range(32) for b in range(w))
+        assert pos == list(range(32 * w))
