@@ -34,10 +34,15 @@ inline bool fwht_fast(const tq_quantizer *q) {
   return q->rotation == TQ_ROT_HADAMARD && (q->d == 32 || q->d == 64 || q->d == 128);
 }
 
+// Validates a row source; *empty is set when n == 0 (a no-op that needs no
+// pointers), in which case TQ_OK is returned before any pointer check.
 tq_status check_rows(const tq_quantizer *q, const void *x, int dtype, int64_t n, int64_t ldx,
-                     const int32_t *chan, int64_t chan_rows) {
-  if (!q || !x || n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_ERR_INVALID_ARG;
+                     const int32_t *chan, int64_t chan_rows, bool *empty = nullptr) {
+  if (!q || n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_ERR_INVALID_ARG;
   if (q->device < 0) return TQ_ERR_UNSUPPORTED;  // host-only quantizer
+  if (empty) *empty = (n == 0);
+  if (n == 0 && empty) return TQ_OK;
+  if (!x) return TQ_ERR_INVALID_ARG;
   if (chan ? chan_rows <= 0 : ldx < q->d) return TQ_ERR_INVALID_ARG;
   if (ldx < 1) return TQ_ERR_INVALID_ARG;
   const size_t es = dtype == TQ_BF16 ? 2 : 4;
@@ -58,15 +63,19 @@ size_t tq_encode_workspace_bytes(const tq_quantizer *q, int64_t n) {
 tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_t n, int64_t ldx,
                        const int32_t *chan, int64_t chan_rows, void *codes, void *signs, float *norms,
                        int64_t out_stride, void *workspace, size_t workspace_bytes, void *stream) {
-  tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows);
-  if (st != TQ_OK) return st;
+  bool empty = false;
+  tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows, &empty);
+  if (st != TQ_OK || empty) return st;
   if (!codes || !signs || !norms || out_stride < 1) return TQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8)) return TQ_ERR_ALIGNMENT;
-  if (n == 0) return TQ_OK;
   DeviceGuard g(q->device);
   if (!g.ok) return TQ_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   RowSource src{x, ldx, chan, chan_rows, q->d, dtype == TQ_BF16};
+  if (tc2_encode_supported(q, dtype, chan != nullptr))
+    return tc2_encode(q, x, n, ldx, codes, signs, norms, out_stride, s);
+  if (tc_encode_supported(q, dtype, ldx, chan != nullptr))
+    return tc_encode(q, x, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, s);
   if (fwht_fast(q)) return v1_encode_fwht(q, src, n, codes, signs, norms, out_stride, s);
   if (!workspace || !aligned(workspace, 16) || v1_dense_batch_rows(q, workspace_bytes) < 1)
     return TQ_ERR_WORKSPACE;
@@ -81,8 +90,9 @@ tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_
   if (ws == 0)
     return tq_encode_ws(q, x, dtype, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, nullptr, 0,
                         stream);
-  tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows);
-  if (st != TQ_OK) return st;
+  bool empty = false;
+  tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows, &empty);
+  if (st != TQ_OK || empty) return st;
   if (!codes || !signs || !norms || out_stride < 1) return TQ_ERR_INVALID_ARG;
   DeviceGuard g(q->device);
   if (!g.ok) return TQ_ERR_CUDA;
@@ -99,11 +109,11 @@ tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_
 
 tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy,
                              const int32_t *ychan, int64_t ychan_rows, float *ytil, float *p, void *stream) {
-  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, ychan_rows);
-  if (st != TQ_OK) return st;
+  bool empty = false;
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, ychan_rows, &empty);
+  if (st != TQ_OK || empty) return st;
   if (!ytil || !p) return TQ_ERR_INVALID_ARG;
   if (!aligned(ytil, 16) || !aligned(p, 16)) return TQ_ERR_ALIGNMENT;
-  if (nq == 0) return TQ_OK;
   DeviceGuard g(q->device);
   if (!g.ok) return TQ_ERR_CUDA;
   RowSource src{y, ldy, ychan, ychan_rows, q->d, 0};
@@ -121,8 +131,9 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_
                    size_t workspace_bytes, void *stream) {
   if (!q || groups < 0 || G < 0 || keys_per_group < 0) return TQ_ERR_INVALID_ARG;
   const int64_t nq = groups * G;
-  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, G > 0 ? G : 1);
-  if (st != TQ_OK) return st;
+  bool empty = false;
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, G > 0 ? G : 1, &empty);
+  if (st != TQ_OK || empty) return st;
   if (!codes || !signs || !norms || !out) return TQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out, 4)) return TQ_ERR_ALIGNMENT;
   if (nq == 0 || keys_per_group == 0) return TQ_OK;
@@ -181,10 +192,10 @@ size_t tq_topk_workspace_bytes(const tq_quantizer *q, int64_t nq, int64_t n, int
 tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy, const void *codes,
                   const void *signs, const float *norms, int64_t n, int k, float *out_scores, int64_t *out_idx,
                   void *workspace, size_t workspace_bytes, void *stream) {
-  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, nullptr, 0);
-  if (st != TQ_OK) return st;
+  bool empty = false;
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, nullptr, 0, &empty);
+  if (st != TQ_OK || empty) return st;
   if (n < 0 || !codes || !signs || !norms || !out_scores || !out_idx) return TQ_ERR_INVALID_ARG;
-  if (nq == 0) return TQ_OK;
   if (k < 1 || k > 64 || k > n) return TQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out_idx, 8) ||
       !aligned(out_scores, 4))

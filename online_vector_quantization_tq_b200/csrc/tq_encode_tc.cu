@@ -1,0 +1,873 @@
+// Tensor-core encode for bf16 keys (d in {32, 64, 96, 128}), one CTA per SM,
+// 256 threads, tiles of 128 vectors.  Per tile:
+//
+//   TMA  x tile (bf16, 128 rows) -> shared memory (double-buffered)
+//   ALU  ||x|| (two threads per row, partial sums exchanged), x * 2^e -> fp16
+//        (exact: bf16 has 8 significant bits) into the A operand tile
+//   MMA  U = X' * Rq^T on tcgen05 (Rq: the rotation as 1 or 2 fp16 pieces;
+//        the Hadamard form d^1.5 R is an integer matrix, exact in fp16), fp32
+//        accumulators in TMEM
+//   ALU  u = U * scale, code = #{t < u}, r = u - c[code] (scaled by 2^10),
+//        gamma^2, r -> fp16 hi + lo into the QJL A operand, codes -> global
+//   MMA  Z = [r_hi | r_lo] * [S | S]^T (S is fp16-exact), fp32 in TMEM
+//   ALU  sign bits of Z -> global (one tile later, overlapping the next
+//        tile's rotation MMA), norms -> global
+//
+// The rotation of tile t runs while the sign bits of tile t-1 are extracted;
+// the QJL projection of tile t runs while tile t+1 is loaded and converted.
+// Method: TurboQuant article 1.2.1-1.2.3 (rotation, Lloyd-Max code, residual,
+// QJL sign sketch), 2.1 (structured rotation), 4.2.1 (stored norm).
+#include <cudaTypedefs.h>
+
+#include "tq_common.cuh"
+#include "tq_kernels.h"
+#include "tq_sm100.cuh"
+
+namespace tq {
+
+struct EncTCParams {
+  int64_t n;
+  int ntiles;
+  const uint16_t *rot16;  // [RP][D][D] fp16 bits, row-major (out, in)
+  const uint16_t *s16;    // [D][D] fp16 bits (QJL rows, in)
+  float rho;              // R = rho * sum of rotation pieces
+  float thr_s[kMaxLevels];   // thresholds * 2^10
+  float cen_s[kMaxLevels];   // centroids * 2^10
+  const int32_t *chan;
+  int64_t chan_rows;
+  uint32_t *codes;
+  uint32_t *signs;
+  float2 *norms;
+  int64_t out_stride;
+  int *err;
+};
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRows = 128;
+constexpr float kRScale = 1024.0f;  // residuals are split into fp16 at 2^10 scale
+
+template <int D, int RP, int SRCW, int NXB>
+struct EncSmem {
+  static constexpr int kXBytes = kRows * SRCW * 2;          // one bf16 x tile (SW128 boxes of 64 cols)
+  static constexpr int kAxBytes = kRows * D * 2;            // fp16 X'
+  static constexpr int kArBytes = kRows * 2 * D * 2;        // fp16 [r_hi | r_lo]
+  static constexpr int kBrBytes = RP * D * D * 2;           // rotation pieces
+  static constexpr int kBsBytes = D * D * 2;                // S
+  static constexpr int kOffX = 0;
+  static constexpr int kOffAx = kOffX + NXB * kXBytes;
+  static constexpr int kOffAr = kOffAx + kAxBytes;
+  static constexpr int kOffBr = kOffAr + kArBytes;
+  static constexpr int kOffBs = kOffBr + kBrBytes;
+  static constexpr int kOffMisc = kOffBs + kBsBytes;
+  static constexpr int kMiscBytes = 4096;
+  static constexpr int kTotal = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+};
+
+// Split of a row's D columns between the two threads of the row: thread half
+// 0 takes [0, SPL), half 1 takes [SPL, D); SPL is a multiple of 32.
+template <int D>
+constexpr int split_point() {
+  return 32 * ((D / 32 + 1) / 2);
+}
+
+// Copy a row-major fp16 [rows][D] matrix from global memory into a 64-byte
+// swizzled K-major operand (D/32 blocks of rows x 64 B).
+template <int D>
+__device__ void stage_kmajor(uint8_t *dst, const uint16_t *src, int rows) {
+  const int chunks = rows * (D / 8);
+  for (int i = threadIdx.x; i < chunks; i += blockDim.x) {
+    const int r = i / (D / 8), c8 = i % (D / 8);  // 8-element chunk index along K
+    const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * D + c8 * 8);
+    const int blk = c8 / 4, ch = c8 % 4;
+    *reinterpret_cast<uint4 *>(dst + (size_t)blk * rows * 64 + sm100::sw64_offset(r, ch)) = v;
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+}  // namespace
+
+template <int D, int W, int RP, int SRCW, int NXB, bool GATHER>
+__global__ void __launch_bounds__(kThreads, 1)
+k_encode_tc(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
+  using SM = EncSmem<D, RP, SRCW, NXB>;
+  constexpr int L = 1 << W;
+  constexpr int SPL = split_point<D>();
+  constexpr int NB = SRCW / 64;  // TMA boxes per x tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sX = smem + SM::kOffX;
+  uint8_t *sAx = smem + SM::kOffAx;
+  uint8_t *sAr = smem + SM::kOffAr;
+  uint8_t *sBr = smem + SM::kOffBr;
+  uint8_t *sBs = smem + SM::kOffBs;
+  float *sRed = reinterpret_cast<float *>(smem + SM::kOffMisc);         // [2][128][2]
+  float *sCen = sRed + 2 * kRows * 2;                                   // [16]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sCen + kMaxLevels);      // full[2], rot, qjl
+  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
+
+  const int tid = threadIdx.x;
+  const int row = tid & (kRows - 1);
+  const int half = tid >> 7;
+  const int c0 = half ? SPL : 0;
+  const int c1 = half ? D : SPL;
+  constexpr int NC0 = SPL, NC1 = D - SPL;
+  const int nc = half ? NC1 : NC0;
+  const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
+
+  // ---- set-up: barriers, TMEM, constant operands
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) sm100::mbar_init(&bars[i], 1);
+    sm100::fence_barrier_init();
+    sm100::prefetch_tmap(&xmap);
+  }
+  if (tid < 32) {
+    sm100::tmem_alloc(sTmem, 256);
+    sm100::tmem_relinquish();
+  }
+  if (tid < kMaxLevels) sCen[tid] = p.cen_s[tid];
+#pragma unroll
+  for (int pc = 0; pc < RP; ++pc) stage_kmajor<D>(sBr + pc * (D * D * 2), p.rot16 + (size_t)pc * D * D, D);
+  stage_kmajor<D>(sBs, p.s16, D);
+  sm100::fence_proxy_async();
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const uint32_t tU = tmem, tZ = tmem + 128;
+  float thr[L - 1];
+#pragma unroll
+  for (int i = 0; i < L - 1; ++i) thr[i] = p.thr_s[i];
+
+  const int first = blockIdx.x;
+  const int stride = gridDim.x;
+  // prefetch the first NXB tiles
+  if (tid == 0) {
+    for (int b = 0; b < NXB; ++b) {
+      const int t = first + b * stride;
+      if (t < p.ntiles) {
+        sm100::mbar_expect_tx(&bars[b], SM::kXBytes);
+        for (int bx = 0; bx < NB; ++bx)
+          sm100::tma_load_2d(sX + b * SM::kXBytes + bx * (kRows * 128), &xmap, bx * 64, t * kRows, &bars[b]);
+      }
+    }
+  }
+
+  uint32_t ph_full[2] = {0u, 0u}, ph_rot = 0u, ph_qjl = 0u;
+  float prev_norm = 0.f, prev_gamma = 0.f;
+  int64_t prev_row = -1;
+  bool failed = false;
+  const uint32_t idesc = sm100::idesc_f16_f32(kRows, D);
+  int it = 0;
+
+  for (int t = first; t < p.ntiles; t += stride, ++it) {
+    const int buf = NXB == 2 ? (it & 1) : 0;
+    const int64_t grow = (int64_t)t * kRows + row;
+    // ---- A: x tile -> registers
+    bool ok = sm100::mbar_wait(&bars[buf], ph_full[buf], p.err, 1);
+    ph_full[buf] ^= 1u;
+    float xv[NC0 > NC1 ? NC0 : NC1];
+    const uint8_t *xt = sX + buf * SM::kXBytes;
+    if constexpr (!GATHER) {
+#pragma unroll
+      for (int k = 0; k < (NC0 > NC1 ? NC0 : NC1) / 8; ++k) {
+        if (k < nc / 8) {
+          const int col = c0 + 8 * k;
+          const uint4 v = *reinterpret_cast<const uint4 *>(xt + (col / 64) * (kRows * 128) +
+                                                           sm100::sw128_offset(row, (col % 64) / 8));
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            xv[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
+            xv[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+          }
+        }
+      }
+    } else {
+      const int32_t *ch = p.chan + (grow / p.chan_rows) * D;
+#pragma unroll
+      for (int j = 0; j < (NC0 > NC1 ? NC0 : NC1); ++j) {
+        if (j < nc) {
+          // masked to the staged tile: a channel index outside the source row
+          // cannot address memory beyond it
+          const int src = grow < p.n ? (__ldg(ch + c0 + j) & (SRCW - 1)) : 0;
+          const uint16_t hv = *reinterpret_cast<const uint16_t *>(
+              xt + (src / 64) * (kRows * 128) + sm100::sw128_offset(row, (src % 64) / 8) + (src % 8) * 2);
+          xv[j] = __uint_as_float((uint32_t)hv << 16);
+        }
+      }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < (NC0 > NC1 ? NC0 : NC1); ++j)
+      if (j < nc) ss = fmaf(xv[j], xv[j], ss);
+    sRed[row * 2 + half] = ss;
+    failed |= __syncthreads_or(!ok) != 0;
+    if (failed) break;
+    // ---- B: norm, scale, fp16 X' -> A operand
+    const float nrm = sqrtf(sRed[row * 2] + sRed[row * 2 + 1]);
+    int e = 0;
+    float s_v = 0.f;  // acc -> u * 2^10
+    if (nrm > 0.f) {
+      e = 14 - (int)((__float_as_uint(nrm) >> 23) & 0xFF) + 127;
+      e = max(-100, min(100, e));
+      s_v = p.rho * kRScale / (nrm * __uint_as_float((uint32_t)(127 + e) << 23));
+    }
+    const float xs = __uint_as_float((uint32_t)(127 + e) << 23);
+#pragma unroll
+    for (int k = 0; k < (NC0 > NC1 ? NC0 : NC1) / 8; ++k) {
+      if (k < nc / 8) {
+        const int col = c0 + 8 * k;
+        uint4 h;
+        h.x = pack_half2(xv[8 * k + 0] * xs, xv[8 * k + 1] * xs);
+        h.y = pack_half2(xv[8 * k + 2] * xs, xv[8 * k + 3] * xs);
+        h.z = pack_half2(xv[8 * k + 4] * xs, xv[8 * k + 5] * xs);
+        h.w = pack_half2(xv[8 * k + 6] * xs, xv[8 * k + 7] * xs);
+        *reinterpret_cast<uint4 *>(sAx + (col / 32) * (kRows * 64) + sm100::sw64_offset(row, (col % 32) / 8)) = h;
+      }
+    }
+    sm100::fence_proxy_async();
+    __syncthreads();
+    // ---- C: rotation MMA; prefetch the tile NXB ahead into this x buffer
+    if (tid == 0) {
+      sm100::tc_fence_after();
+      const uint32_t ax = sm100::smem_u32(sAx), br = sm100::smem_u32(sBr);
+#pragma unroll
+      for (int pc = 0; pc < RP; ++pc)
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t a = sm100::desc_sw64(ax + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+          const uint64_t b = sm100::desc_sw64(br + pc * (D * D * 2) + (ks >> 1) * (D * 64) + (ks & 1) * 32);
+          sm100::mma_f16(tU, a, b, idesc, (pc | ks) != 0);
+        }
+      sm100::mma_commit(&bars[2]);
+      const int tn = t + NXB * stride;
+      if (tn < p.ntiles) {
+        sm100::mbar_expect_tx(&bars[buf], SM::kXBytes);
+        for (int bx = 0; bx < NB; ++bx)
+          sm100::tma_load_2d(sX + buf * SM::kXBytes + bx * (kRows * 128), &xmap, bx * 64, tn * kRows, &bars[buf]);
+      }
+    }
+    // ---- D: sign bits of the previous tile
+    if (it > 0) {
+      ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 3);
+      ph_qjl ^= 1u;
+      sm100::tc_fence_after();
+#pragma unroll
+      for (int g = 0; g < (NC0 > NC1 ? NC0 : NC1) / 32; ++g) {
+        if (g < nc / 32) {
+          uint32_t z[32];
+          sm100::tmem_ld16(tZ + lane_base + c0 + 32 * g, *reinterpret_cast<uint32_t(*)[16]>(&z[0]));
+          sm100::tmem_ld16(tZ + lane_base + c0 + 32 * g + 16, *reinterpret_cast<uint32_t(*)[16]>(&z[16]));
+          sm100::tmem_wait_ld();
+          uint32_t wbits = 0u;
+#pragma unroll
+          for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+          if (prev_row >= 0 && prev_row < p.n)
+            p.signs[prev_row * p.out_stride * (D / 32) + (c0 / 32) + g] = ~wbits;
+        }
+      }
+      if (half == 0 && prev_row >= 0 && prev_row < p.n)
+        p.norms[prev_row * p.out_stride] = make_float2(prev_norm, prev_gamma);
+    }
+    // ---- E: rotated coordinates -> codes, residual split
+    ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 2) && ok;
+    ph_rot ^= 1u;
+    sm100::tc_fence_after();
+    float g2 = 0.f;
+#pragma unroll
+    for (int g = 0; g < (NC0 > NC1 ? NC0 : NC1) / 32; ++g) {
+      if (g < nc / 32) {
+        uint32_t acc[32];
+        sm100::tmem_ld16(tU + lane_base + c0 + 32 * g, *reinterpret_cast<uint32_t(*)[16]>(&acc[0]));
+        sm100::tmem_ld16(tU + lane_base + c0 + 32 * g + 16, *reinterpret_cast<uint32_t(*)[16]>(&acc[16]));
+        sm100::tmem_wait_ld();
+        uint32_t cw[W];
+#pragma unroll
+        for (int k = 0; k < W; ++k) cw[k] = 0u;
+        float rs[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float us = __uint_as_float(acc[j]) * s_v;
+          int c = 0;
+#pragma unroll
+          for (int i = 0; i < L - 1; ++i) c += us > thr[i] ? 1 : 0;
+          pack_code<W>(cw, j, (uint32_t)c);
+          rs[j] = us - sCen[c];
+          g2 = fmaf(rs[j], rs[j], g2);
+        }
+        if (grow < p.n) {
+          uint32_t *dst = p.codes + grow * p.out_stride * (W * D / 32) + ((c0 / 32) + g) * W;
+#pragma unroll
+          for (int k = 0; k < W; ++k) dst[k] = cw[k];
+        }
+        // r = hi + lo, both fp16, into [r_hi | r_lo]
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float a = rs[8 * k + 2 * e2], b = rs[8 * k + 2 * e2 + 1];
+            const __half2 h = __floats2half2_rn(a, b);
+            const float2 hf = __half22float2(h);
+            hi[e2] = *reinterpret_cast<const uint32_t *>(&h);
+            lo[e2] = pack_half2(a - hf.x, b - hf.y);
+          }
+          const int col = c0 + 32 * g + 8 * k;
+          *reinterpret_cast<uint4 *>(sAr + (col / 32) * (kRows * 64) + sm100::sw64_offset(row, (col % 32) / 8)) =
+              make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(sAr + ((D + col) / 32) * (kRows * 64) +
+                                     sm100::sw64_offset(row, (col % 32) / 8)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+    }
+    sRed[2 * kRows + row * 2 + half] = g2;
+    sm100::fence_proxy_async();
+    sm100::tc_fence_before();
+    failed |= __syncthreads_or(!ok) != 0;
+    if (failed) break;
+    // ---- F: QJL MMA
+    if (tid == 0) {
+      sm100::tc_fence_after();
+      const uint32_t ar = sm100::smem_u32(sAr), bs = sm100::smem_u32(sBs);
+#pragma unroll
+      for (int ks = 0; ks < 2 * D / 16; ++ks) {
+        const int kk = ks % (D / 16);
+        const uint64_t a = sm100::desc_sw64(ar + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+        const uint64_t b = sm100::desc_sw64(bs + (kk >> 1) * (D * 64) + (kk & 1) * 32);
+        sm100::mma_f16(tZ, a, b, idesc, ks != 0);
+      }
+      sm100::mma_commit(&bars[3]);
+    }
+    prev_norm = nrm;
+    prev_gamma = sqrtf(sRed[2 * kRows + row * 2] + sRed[2 * kRows + row * 2 + 1]) * (1.0f / kRScale);
+    prev_row = grow;
+  }
+
+  // ---- drain: sign bits of the last tile
+  if (!failed && it > 0) {
+    const bool ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 4);
+    sm100::tc_fence_after();
+    if (ok) {
+#pragma unroll
+      for (int g = 0; g < (NC0 > NC1 ? NC0 : NC1) / 32; ++g) {
+        if (g < nc / 32) {
+          uint32_t z[32];
+          sm100::tmem_ld16(tZ + lane_base + c0 + 32 * g, *reinterpret_cast<uint32_t(*)[16]>(&z[0]));
+          sm100::tmem_ld16(tZ + lane_base + c0 + 32 * g + 16, *reinterpret_cast<uint32_t(*)[16]>(&z[16]));
+          sm100::tmem_wait_ld();
+          uint32_t wbits = 0u;
+#pragma unroll
+          for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+          if (prev_row >= 0 && prev_row < p.n)
+            p.signs[prev_row * p.out_stride * (D / 32) + (c0 / 32) + g] = ~wbits;
+        }
+      }
+      if (half == 0 && prev_row >= 0 && prev_row < p.n)
+        p.norms[prev_row * p.out_stride] = make_float2(prev_norm, prev_gamma);
+    }
+  }
+  if (failed && tid == 0) {
+    // bounded wait for x-tile loads still in flight before the CTA exits
+    for (int b = 0; b < NXB; ++b) sm100::mbar_wait(&bars[b], ph_full[b], p.err, 5);
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (tid < 32) sm100::tmem_dealloc(tmem, 256);
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+template <int D, int W, int RP, int SRCW, bool GATHER>
+tq_status launch_tc(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, int64_t cols,
+                    const EncTCParams &prm, cudaStream_t st) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return TQ_ERR_CUDA;
+  CUtensorMap map;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)n};
+  cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), gdim, gstride, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return TQ_ERR_CUDA;
+  int dev = 0, max_smem = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntiles = (int)((n + kRows - 1) / kRows);
+  EncTCParams pp = prm;
+  pp.ntiles = ntiles;
+  const int grid = std::min(ntiles, sms);
+  if (EncSmem<D, RP, SRCW, 2>::kTotal <= max_smem) {
+    auto kern = k_encode_tc<D, W, RP, SRCW, 2, GATHER>;
+    const int sm = EncSmem<D, RP, SRCW, 2>::kTotal;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    kern<<<grid, kThreads, sm, st>>>(map, pp);
+  } else {
+    auto kern = k_encode_tc<D, W, RP, SRCW, 1, GATHER>;
+    const int sm = EncSmem<D, RP, SRCW, 1>::kTotal;
+    if (sm > max_smem) return TQ_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    kern<<<grid, kThreads, sm, st>>>(map, pp);
+  }
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+template <int D, int W, int RP>
+tq_status dispatch_src(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, bool gather,
+                       const EncTCParams &prm, cudaStream_t st) {
+  if (gather) return launch_tc<D, W, RP, 128, true>(q, x, n, ldx, ldx, prm, st);
+  constexpr int SW = (D + 63) / 64 * 64;
+  return launch_tc<D, W, RP, SW, false>(q, x, n, ldx, D, prm, st);
+}
+
+template <int D, int W>
+tq_status dispatch_rp(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, bool gather,
+                      const EncTCParams &prm, cudaStream_t st) {
+  if (q->tc_rot_pieces == 1) return dispatch_src<D, W, 1>(q, x, n, ldx, gather, prm, st);
+  return dispatch_src<D, W, 2>(q, x, n, ldx, gather, prm, st);
+}
+
+template <int D>
+tq_status dispatch_w(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, bool gather,
+                     const EncTCParams &prm, cudaStream_t st) {
+  switch (q->w) {
+    case 1: return dispatch_rp<D, 1>(q, x, n, ldx, gather, prm, st);
+    case 2: return dispatch_rp<D, 2>(q, x, n, ldx, gather, prm, st);
+    case 3: return dispatch_rp<D, 3>(q, x, n, ldx, gather, prm, st);
+    case 4: return dispatch_rp<D, 4>(q, x, n, ldx, gather, prm, st);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+bool tc_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather) {
+  if (dtype != TQ_BF16 || !q->d_rot16 || q->tc_rot_pieces < 1) return false;
+  const int d = q->d;
+  if (d != 32 && d != 64 && d != 96 && d != 128) return false;
+  if (d == 128 && q->tc_rot_pieces > 1) return false;  // operands would exceed shared memory
+  if (gather) return ldx <= 128 && ldx >= 64 && ldx % 64 == 0;
+  return d >= 64;  // a 32-column tile would be narrower than the 64-column load box
+}
+
+tq_status tc_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,
+                    int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,
+                    cudaStream_t st) {
+  EncTCParams prm{};
+  prm.n = n;
+  prm.rot16 = q->d_rot16;
+  prm.s16 = q->d_qjl16;
+  prm.rho = q->tc_rho;
+  for (int i = 0; i < kMaxLevels; ++i) {
+    prm.thr_s[i] = q->kt.thresholds[i] * kRScale;
+    prm.cen_s[i] = q->kt.centroids[i] * kRScale;
+  }
+  prm.chan = chan;
+  prm.chan_rows = chan_rows;
+  prm.codes = static_cast<uint32_t *>(codes);
+  prm.signs = static_cast<uint32_t *>(signs);
+  prm.norms = reinterpret_cast<float2 *>(norms);
+  prm.out_stride = out_stride;
+  prm.err = q->d_err;
+  const bool gather = chan != nullptr;
+  switch (q->d) {
+    case 32: return dispatch_w<32>(q, x, n, ldx, gather, prm, st);
+    case 64: return dispatch_w<64>(q, x, n, ldx, gather, prm, st);
+    case 96: return dispatch_w<96>(q, x, n, ldx, gather, prm, st);
+    case 128: return dispatch_w<128>(q, x, n, ldx, gather, prm, st);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace tq
+
+namespace tq {
+
+// ============================================================================
+// Encode for bf16 keys with the Hadamard rotation, reading the TMA tile as
+// the MMA's A operand directly (no conversion on the CUDA cores).
+//
+//   d^1.5 R = K is an integer matrix; K = K_hi + K_lo with both pieces exact
+//   in bf16, so U = X K^T takes two bf16 MMA passes and is exact up to fp32
+//   accumulation.  R is orthogonal, so ||x|| = ||U|| / d^1.5 and
+//   u = U / ||U||: the norm comes from the rotated row.
+//
+// 128 * (d/32) threads; thread (row, p) owns columns [32p, 32p+32) of one
+// row.  Per-row partial sums (||U||^2, gamma^2) go through four spare TMEM
+// columns.  The rotation of tile t+1 is issued before the residuals of tile
+// t are computed (U is double-buffered in TMEM), and the sign bits of tile
+// t-1 are read while the QJL projection of tile t is being prepared.
+// ============================================================================
+namespace {
+
+template <int D>
+struct Enc2Smem {
+  static constexpr int kXBytes = kRows * D * 2;
+  static constexpr int kOffX = 0;                       // 2 x tiles (TMA, 128-byte swizzle)
+  static constexpr int kOffAr = 2 * kXBytes;            // [r_hi | r_lo] fp16, 64-byte swizzle
+  static constexpr int kOffBr = kOffAr + kRows * 2 * D * 2;  // K_hi, K_lo bf16
+  static constexpr int kOffBs = kOffBr + 2 * D * D * 2;      // S fp16
+  static constexpr int kOffMisc = kOffBs + D * D * 2;
+  static constexpr int kTotal = kOffMisc + 128 + 1024;
+};
+
+}  // namespace
+
+template <int D, int W>
+__global__ void __launch_bounds__(128 * (D / 32), 1)
+k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
+  constexpr int P = D / 32;
+  constexpr int L = 1 << W;
+  constexpr int HALF = L / 2;
+  constexpr int NB = D / 64;  // TMA boxes of 64 columns
+  constexpr uint32_t kColU0 = 0, kColZ = 256, kColScr = 384;
+  using SM = Enc2Smem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sX = smem + SM::kOffX;
+  uint8_t *sAr = smem + SM::kOffAr;
+  uint8_t *sBr = smem + SM::kOffBr;
+  uint8_t *sBs = smem + SM::kOffBs;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffMisc);  // full[2], rot, qjl
+  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
+
+  const int tid = threadIdx.x;
+  const int row = tid & (kRows - 1);
+  const int pc = tid >> 7;  // column group
+  const uint32_t lane = (uint32_t)(row & ~31) << 16;
+
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) sm100::mbar_init(&bars[i], 1);
+    sm100::fence_barrier_init();
+    sm100::prefetch_tmap(&xmap);
+  }
+  if (tid < 32) {
+    sm100::tmem_alloc(sTmem, 512);
+    sm100::tmem_relinquish();
+  }
+  stage_kmajor<D>(sBr, p.rot16, D);
+  stage_kmajor<D>(sBr + D * D * 2, p.rot16 + (size_t)D * D, D);
+  stage_kmajor<D>(sBs, p.s16, D);
+  sm100::fence_proxy_async();
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+
+  // Symmetric codebook (scaled 2^10): magnitude thresholds T_k, k = 1..HALF-1,
+  // and centroid magnitudes C_k.  Each threshold test is the exact step
+  // sat(2^40 (u^2 - T_k^2)): fp32 values that differ do so by far more than
+  // 2^-40, so the step is exactly 0 or 1 (u^2 vs the rounded T_k^2 can only
+  // disagree with |u| vs T_k within an ulp of the threshold).
+  constexpr float kBig = 1099511627776.0f;  // 2^40
+  float nT2B[HALF], dC[HALF];
+#pragma unroll
+  for (int k = 0; k < HALF; ++k) {
+    const float tk = p.thr_s[HALF - 1 + k];
+    nT2B[k] = -(tk * tk) * kBig;
+    dC[k] = k == 0 ? p.cen_s[HALF] : p.cen_s[HALF + k] - p.cen_s[HALF + k - 1];
+  }
+
+  const uint32_t idesc_rot = sm100::idesc_bf16_f32(kRows, D);
+  const uint32_t idesc_qjl = sm100::idesc_f16_f32(kRows, D);
+  const int first = blockIdx.x, stride = gridDim.x;
+
+  auto issue_rot = [&](int buf, uint32_t ucol) {
+    const uint32_t xa = sm100::smem_u32(sX + buf * SM::kXBytes), br = sm100::smem_u32(sBr);
+#pragma unroll
+    for (int piece = 0; piece < 2; ++piece)
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t a = sm100::desc_sw128(xa + (ks >> 2) * (kRows * 128) + (ks & 3) * 32);
+        const uint64_t b = sm100::desc_sw64(br + piece * (D * D * 2) + (ks >> 1) * (D * 64) + (ks & 1) * 32);
+        sm100::mma_f16(tmem + ucol, a, b, idesc_rot, (piece | ks) != 0);
+      }
+    sm100::mma_commit(&bars[2]);
+  };
+  auto issue_tma = [&](int buf, int tile) {
+    sm100::mbar_expect_tx(&bars[buf], SM::kXBytes);
+#pragma unroll
+    for (int bx = 0; bx < NB; ++bx)
+      sm100::tma_load_2d(sX + buf * SM::kXBytes + bx * (kRows * 128), &xmap, bx * 64, tile * kRows, &bars[buf]);
+  };
+
+  // thread 0's bookkeeping of asynchronous work in flight
+  bool pend_full[2] = {false, false};
+  uint32_t ph_full[2] = {0u, 0u};
+  bool failed = false;
+  if (tid == 0 && first < p.ntiles) {
+    issue_tma(0, first);
+    pend_full[0] = true;
+    if (first + stride < p.ntiles) {
+      issue_tma(1, first + stride);
+      pend_full[1] = true;
+    }
+    if (!sm100::mbar_wait(&bars[0], ph_full[0], p.err, 11)) failed = true;
+    ph_full[0] ^= 1u;
+    pend_full[0] = false;
+    sm100::tc_fence_after();
+    if (!failed) issue_rot(0, kColU0);
+  }
+
+  uint32_t ph_rot = 0u, ph_qjl = 0u;
+  float prev_norm = 0.f, prev_gamma = 0.f;
+  int64_t prev_row = -1;
+  int it = 0;
+  for (int t = first; t < p.ntiles; t += stride, ++it) {
+    const int buf = it & 1;
+    const int64_t grow = (int64_t)t * kRows + row;
+    const uint32_t ucol = (it & 1) ? 128u : 0u;
+    // ---- (1) rotated tile -> registers, ||U||^2 partial -> TMEM scratch
+    bool ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 12);
+    ph_rot ^= 1u;
+    sm100::tc_fence_after();
+    uint32_t acc[32];
+    sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
+    sm100::tmem_wait_ld();
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ss = fmaf(__uint_as_float(acc[j]), __uint_as_float(acc[j]), ss);
+    sm100::tmem_st1(tmem + lane + kColScr + pc, __float_as_uint(ss));
+    sm100::tmem_wait_st();
+    sm100::tc_fence_before();
+    failed |= __syncthreads_or(!ok || failed) != 0;
+    if (failed) break;
+    sm100::tc_fence_after();
+    if (tid == 0) {
+      // x tile t has been consumed: refill this buffer, start the next rotation
+      const int t2 = t + 2 * stride;
+      if (t2 < p.ntiles) {
+        issue_tma(buf, t2);
+        pend_full[buf] = true;
+      }
+      const int t1 = t + stride;
+      if (t1 < p.ntiles) {
+        const int b1 = buf ^ 1;
+        if (!sm100::mbar_wait(&bars[b1], ph_full[b1], p.err, 13)) failed = true;
+        ph_full[b1] ^= 1u;
+        pend_full[b1] = false;
+        sm100::tc_fence_after();
+        if (!failed) issue_rot(b1, ucol ^ 128u);
+      }
+    }
+    // ---- (3a) norm, codes, residual split (kept in registers)
+    uint32_t parts[4];
+    sm100::tmem_ld4(tmem + lane + kColScr, parts);
+    sm100::tmem_wait_ld();
+    float nacc = 0.f;
+#pragma unroll
+    for (int k = 0; k < P; ++k) nacc += __uint_as_float(parts[k]);
+    nacc = sqrtf(nacc);
+    const float nrm = nacc * p.rho;
+    const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;  // zero rows: u = -0 -> lower middle code
+    uint32_t cw[W];
+#pragma unroll
+    for (int k = 0; k < W; ++k) cw[k] = 0u;
+    uint32_t hi[16], lo[16];
+    float g2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      float rr[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float us = __uint_as_float(acc[j + e]) * s_v;
+        const float usb = us * kBig;
+        float cm = dC[0], m = 0.f;
+#pragma unroll
+        for (int k = 1; k < HALF; ++k) {
+          const float st = __saturatef(__fmaf_rn(us, usb, nT2B[k]));
+          cm = __fmaf_rn(st, dC[k], cm);
+          m += st;
+        }
+        // s = +-1 from the sign bit (u = -0 takes the lower middle code)
+        const float sg = __uint_as_float((__float_as_uint(us) & 0x80000000u) | 0x3F800000u);
+        const float s01 = __fmaf_rn(sg, 0.5f, 0.5f);
+        // code = HALF-1+s01 + s*m, as the low bits of 2^23 + code
+        const float codef = __fmaf_rn(sg, m, s01 + (8388608.0f + (float)(HALF - 1)));
+        rr[e] = __fmaf_rn(-sg, cm, us);
+        pack_code<W>(cw, j + e, __float_as_uint(codef) & (uint32_t)(L - 1));
+        g2 = fmaf(rr[e], rr[e], g2);
+      }
+      const __half2 h = __floats2half2_rn(rr[0], rr[1]);
+      const float2 hf = __half22float2(h);
+      hi[j / 2] = *reinterpret_cast<const uint32_t *>(&h);
+      lo[j / 2] = pack_half2(rr[0] - hf.x, rr[1] - hf.y);
+    }
+    if (grow < p.n) {
+      uint32_t *dst = p.codes + grow * p.out_stride * (W * D / 32) + pc * W;
+#pragma unroll
+      for (int k = 0; k < W; ++k) dst[k] = cw[k];
+    }
+    // ---- (2) sign bits of the previous tile
+    if (it > 0) {
+      ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 14) && ok;
+      ph_qjl ^= 1u;
+      sm100::tc_fence_after();
+      uint32_t z[32];
+      sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+      sm100::tmem_wait_ld();
+      uint32_t wbits = 0u;
+#pragma unroll
+      for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+      if (prev_row >= 0 && prev_row < p.n) {
+        p.signs[prev_row * p.out_stride * (D / 32) + pc] = ~wbits;
+        if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, prev_gamma);
+      }
+    }
+    // ---- (3b) residual operand, gamma^2 partial
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      *reinterpret_cast<uint4 *>(sAr + pc * (kRows * 64) + sm100::sw64_offset(row, k)) =
+          make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
+      *reinterpret_cast<uint4 *>(sAr + (P + pc) * (kRows * 64) + sm100::sw64_offset(row, k)) =
+          make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+    }
+    sm100::tmem_st1(tmem + lane + kColScr + 4 + pc, __float_as_uint(g2));
+    sm100::tmem_wait_st();
+    sm100::fence_proxy_async();
+    sm100::tc_fence_before();
+    failed |= __syncthreads_or(!ok || failed) != 0;
+    if (failed) break;
+    sm100::tc_fence_after();
+    // ---- (4) QJL projection of this tile
+    if (tid == 0) {
+      const uint32_t ar = sm100::smem_u32(sAr), bs = sm100::smem_u32(sBs);
+#pragma unroll
+      for (int ks = 0; ks < 2 * D / 16; ++ks) {
+        const int kk = ks % (D / 16);
+        const uint64_t a = sm100::desc_sw64(ar + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+        const uint64_t b = sm100::desc_sw64(bs + (kk >> 1) * (D * 64) + (kk & 1) * 32);
+        sm100::mma_f16(tmem + kColZ, a, b, idesc_qjl, ks != 0);
+      }
+      sm100::mma_commit(&bars[3]);
+    }
+    float gsum = 0.f;
+    if (pc == 0) {
+      sm100::tmem_ld4(tmem + lane + kColScr + 4, parts);
+      sm100::tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < P; ++k) gsum += __uint_as_float(parts[k]);
+    }
+    prev_norm = nrm;
+    prev_gamma = sqrtf(gsum) * (1.0f / kRScale);
+    prev_row = grow;
+  }
+
+  // ---- drain: sign bits of the last tile
+  if (!failed && it > 0) {
+    const bool ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 15);
+    sm100::tc_fence_after();
+    if (ok) {
+      uint32_t z[32];
+      sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+      sm100::tmem_wait_ld();
+      uint32_t wbits = 0u;
+#pragma unroll
+      for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+      if (prev_row >= 0 && prev_row < p.n) {
+        p.signs[prev_row * p.out_stride * (D / 32) + pc] = ~wbits;
+        if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, prev_gamma);
+      }
+    }
+  }
+  if (failed && tid == 0) {
+    for (int b = 0; b < 2; ++b)
+      if (pend_full[b]) sm100::mbar_wait(&bars[b], ph_full[b], p.err, 16);
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (tid < 32) sm100::tmem_dealloc(tmem, 512);
+}
+
+namespace {
+template <int D, int W>
+tq_status launch_tc2(const void *x, int64_t n, int64_t ldx, const EncTCParams &prm, cudaStream_t st) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return TQ_ERR_CUDA;
+  CUtensorMap map;
+  cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)n};
+  cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), gdim, gstride, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return TQ_ERR_CUDA;
+  int dev = 0, max_smem = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  constexpr int smem = Enc2Smem<D>::kTotal;
+  if (smem > max_smem) return TQ_ERR_UNSUPPORTED;
+  EncTCParams pp = prm;
+  pp.ntiles = (int)((n + kRows - 1) / kRows);
+  auto kern = k_encode_tc2<D, W>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32), smem, st>>>(map, pp);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+}  // namespace
+
+bool tc2_encode_supported(const tq_quantizer *q, int dtype, bool gather) {
+  return dtype == TQ_BF16 && !gather && q->d_rot_bf16 && (q->d == 64 || q->d == 128);
+}
+
+tq_status tc2_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, void *codes, void *signs,
+                     float *norms, int64_t out_stride, cudaStream_t st) {
+  EncTCParams prm{};
+  prm.n = n;
+  prm.rot16 = q->d_rot_bf16;
+  prm.s16 = q->d_qjl16;
+  prm.rho = q->tc_rho;
+  for (int i = 0; i < kMaxLevels; ++i) {
+    prm.thr_s[i] = q->kt.thresholds[i] * kRScale;
+    prm.cen_s[i] = q->kt.centroids[i] * kRScale;
+  }
+  prm.codes = static_cast<uint32_t *>(codes);
+  prm.signs = static_cast<uint32_t *>(signs);
+  prm.norms = reinterpret_cast<float2 *>(norms);
+  prm.out_stride = out_stride;
+  prm.err = q->d_err;
+#define TQ_TC2(DD)                                                        \
+  switch (q->w) {                                                         \
+    case 1: return launch_tc2<DD, 1>(x, n, ldx, prm, st);                 \
+    case 2: return launch_tc2<DD, 2>(x, n, ldx, prm, st);                 \
+    case 3: return launch_tc2<DD, 3>(x, n, ldx, prm, st);                 \
+    case 4: return launch_tc2<DD, 4>(x, n, ldx, prm, st);                 \
+  }                                                                       \
+  return TQ_ERR_UNSUPPORTED;
+  if (q->d == 64) {
+    TQ_TC2(64)
+  }
+  if (q->d == 128) {
+    TQ_TC2(128)
+  }
+#undef TQ_TC2
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace tq

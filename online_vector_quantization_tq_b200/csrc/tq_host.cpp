@@ -252,6 +252,12 @@ tq_status upload(T **dst, const T *src, size_t count) {
 }
 
 void free_device(tq_quantizer *q) {
+  cudaFree(q->d_rot16);
+  cudaFree(q->d_rot_bf16);
+  cudaFree(q->d_err);
+  q->d_rot16 = nullptr;
+  q->d_rot_bf16 = nullptr;
+  q->d_err = nullptr;
   cudaFree(q->d_diag_bits);
   cudaFree(q->d_rot);
   cudaFree(q->d_qjl16);
@@ -370,6 +376,7 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
       for (int i = 0; i < d; ++i) cur[(size_t)i * d + j] = col[i];
     }
     for (size_t i = 0; i < cur.size(); ++i) q->rot[i] = (float)cur[i];
+    q->rot_exact = cur;
   } else {
     std::vector<double> h;
     haar(d, seed, h);
@@ -401,6 +408,71 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
   if (st == TQ_OK) st = upload(&q->d_rot, q->rot.data(), q->rot.size());
   if (st == TQ_OK) st = upload(&q->d_qjl16, q->qjl16.data(), q->qjl16.size());
   if (st == TQ_OK) st = upload(&q->d_qjl32, s32.data(), s32.size());
+  if (st == TQ_OK) {
+    // Rotation as fp16 pieces for the tensor-core encode.  Hadamard: d^1.5 R
+    // is an integer matrix (exact in fp16 when every |entry| <= 2048, else
+    // split into two exact pieces).  Haar: R * 2^8 split into hi + lo fp16.
+    std::vector<uint16_t> pieces;
+    const size_t dd = (size_t)d * d;
+    if (rot == TQ_ROT_HADAMARD) {
+      const double s15 = std::pow((double)d, 1.5);
+      double big = 0.0;
+      std::vector<double> kmat(dd);
+      for (size_t i = 0; i < dd; ++i) {
+        kmat[i] = std::nearbyint((double)q->rot_exact[i] * s15);
+        big = std::max(big, std::fabs(kmat[i]));
+      }
+      q->tc_rho = (float)(1.0 / s15);
+      q->tc_rot_pieces = big <= 2048.0 ? 1 : 2;
+      pieces.resize(q->tc_rot_pieces * dd);
+      for (size_t i = 0; i < dd; ++i) {
+        const uint16_t h = double_to_half_bits(kmat[i]);
+        pieces[i] = h;
+        if (q->tc_rot_pieces == 2) pieces[dd + i] = double_to_half_bits(kmat[i] - half_bits_to_double(h));
+      }
+      if (big <= 2048.0) {
+        // the same integer matrix as two bf16 pieces (8 + 8 significant bits
+        // cover integers up to 2^11 exactly), for MMAs that read bf16 keys as-is
+        std::vector<uint16_t> bfp(2 * dd);
+        auto to_bf16 = [](double v) {
+          float f = (float)v;  // exact: an integer below 2^24
+          uint32_t b;
+          std::memcpy(&b, &f, 4);
+          b += 0x7FFFu + ((b >> 16) & 1u);
+          return (uint16_t)(b >> 16);
+        };
+        auto from_bf16 = [](uint16_t h) {
+          uint32_t b = (uint32_t)h << 16;
+          float f;
+          std::memcpy(&f, &b, 4);
+          return (double)f;
+        };
+        for (size_t i = 0; i < dd; ++i) {
+          const uint16_t h = to_bf16(kmat[i]);
+          bfp[i] = h;
+          bfp[dd + i] = to_bf16(kmat[i] - from_bf16(h));
+        }
+        st = upload(&q->d_rot_bf16, bfp.data(), bfp.size());
+      }
+    } else {
+      q->tc_rho = 1.0f / 256.0f;
+      q->tc_rot_pieces = 2;
+      pieces.resize(2 * dd);
+      for (size_t i = 0; i < dd; ++i) {
+        const double v = (double)q->rot[i] * 256.0;
+        const uint16_t h = double_to_half_bits(v);
+        pieces[i] = h;
+        pieces[dd + i] = double_to_half_bits(v - half_bits_to_double(h));
+      }
+    }
+    if (st == TQ_OK) st = upload(&q->d_rot16, pieces.data(), pieces.size());
+  }
+  if (st == TQ_OK) {
+    if (cudaMalloc((void **)&q->d_err, sizeof(int)) != cudaSuccess || cudaMemset(q->d_err, 0, sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      st = TQ_ERR_NOMEM;
+    }
+  }
   if (st != TQ_OK) {
     free_device(q);
     delete q;

@@ -32,6 +32,7 @@ struct tq_quantizer {
   std::vector<double> centroids, thresholds;
   double coord_mse = 0.0;
   std::vector<float> rot;        // d x d fp32 (Haar, or the dense Hadamard product)
+  std::vector<double> rot_exact; // d x d double (Hadamard product; empty for Haar)
   std::vector<int8_t> diag;      // 3 x d (Hadamard)
   std::vector<uint16_t> qjl16;   // m x d fp16 bits
   // device copies (owned)
@@ -39,6 +40,12 @@ struct tq_quantizer {
   float *d_rot = nullptr;
   uint16_t *d_qjl16 = nullptr;
   float *d_qjl32 = nullptr;
+  // tensor-core encode: R = tc_rho * (sum of tc_rot_pieces fp16 matrices)
+  uint16_t *d_rot16 = nullptr;   // [pieces][d][d] fp16 bits
+  int tc_rot_pieces = 0;
+  float tc_rho = 0.f;
+  uint16_t *d_rot_bf16 = nullptr;  // Hadamard: d^1.5 R as two exact bf16 pieces [2][d][d]
+  int *d_err = nullptr;          // device error word (bounded waits that timed out)
   tq::KernelTables kt{};
 };
 

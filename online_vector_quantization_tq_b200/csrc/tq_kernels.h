@@ -26,4 +26,13 @@ tq_status v1_topk_select(float *score, const int64_t *idx, int64_t rows, int64_t
 tq_status v1_sumsq(const RowSource &src, int64_t groups, int64_t rows_per_group, double *part, int nchunks,
                    double *out, cudaStream_t st);
 
+bool tc_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather);
+tq_status tc_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,
+                    int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,
+                    cudaStream_t st);
+
+bool tc2_encode_supported(const tq_quantizer *q, int dtype, bool gather);
+tq_status tc2_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, void *codes, void *signs,
+                     float *norms, int64_t out_stride, cudaStream_t st);
+
 }  // namespace tq
