@@ -120,9 +120,29 @@ tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq, 
   return v1_prepare_queries(q, src, nq, ytil, p, static_cast<cudaStream_t>(stream));
 }
 
+// Workspace of tq_score: prepared queries (y~, p), then the integer scorer's
+// query operand (at most 16 rows of 384 bytes per query) and per-query scales.
+struct ScoreLayout {
+  size_t ytil, p, qop, qsc, total;
+};
+ScoreLayout score_layout(const tq_quantizer *q, int64_t nq) {
+  ScoreLayout L{};
+  size_t off = 0;
+  L.ytil = off;
+  off += round_up((size_t)nq * q->d * 4, 256);
+  L.p = off;
+  off += round_up((size_t)nq * q->m * 4, 256);
+  L.qop = off;
+  off += round_up((size_t)nq * 16 * 384, 256);
+  L.qsc = off;
+  off += round_up((size_t)nq * 16, 256);
+  L.total = off;
+  return L;
+}
+
 size_t tq_score_workspace_bytes(const tq_quantizer *q, int64_t nq) {
   if (!q || nq <= 0) return 0;
-  return round_up((size_t)nq * q->d * 4, 256) + round_up((size_t)nq * q->m * 4, 256);
+  return score_layout(q, nq).total;
 }
 
 tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_t G, int64_t ldy,
@@ -142,11 +162,17 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_
   DeviceGuard g(q->device);
   if (!g.ok) return TQ_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float *ytil = static_cast<float *>(workspace);
-  float *p = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up((size_t)nq * q->d * 4, 256));
+  const ScoreLayout L = score_layout(q, nq);
+  char *ws = static_cast<char *>(workspace);
+  float *ytil = reinterpret_cast<float *>(ws + L.ytil);
+  float *p = reinterpret_cast<float *>(ws + L.p);
   RowSource src{y, ldy, ychan, G, q->d, 0};
   st = v1_prepare_queries(q, src, nq, ytil, p, s);
   if (st != TQ_OK) return st;
+  if (tc_score_supported(q, G) && aligned(codes, 16) && aligned(signs, 16))
+    return tc_score(q, ytil, p, groups, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
+                    keys_per_group, accumulate, reinterpret_cast<int8_t *>(ws + L.qop),
+                    reinterpret_cast<float4 *>(ws + L.qsc), s);
   return v1_score(q, ytil, p, nq, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
                   keys_per_group, accumulate, s);
 }
@@ -158,7 +184,7 @@ constexpr int64_t kTopkChunk = 65536;
 constexpr int64_t kTopkSlice = 2048;
 
 struct TopkLayout {
-  size_t ytil, p, scores, part_s, part_i, total;
+  size_t ytil, p, qop, qsc, scores, part_s, part_i, total;
   int64_t chunk, nparts;
 };
 
@@ -171,6 +197,10 @@ TopkLayout topk_layout(const tq_quantizer *q, int64_t nq, int64_t n, int k) {
   off += round_up((size_t)nq * q->d * 4, 256);
   L.p = off;
   off += round_up((size_t)nq * q->m * 4, 256);
+  L.qop = off;
+  off += round_up((size_t)std::min<int64_t>(nq, 48) * 16 * 384, 256);
+  L.qsc = off;
+  off += round_up((size_t)nq * 16, 256);
   L.scores = off;
   off += round_up((size_t)nq * L.chunk * 4, 256);
   L.part_s = off;
@@ -214,9 +244,20 @@ tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy
   RowSource src{y, ldy, nullptr, 0, q->d, 0};
   st = v1_prepare_queries(q, src, nq, ytil, p, s);
   if (st != TQ_OK) return st;
+  const bool tc = tc_score_supported(q, std::min<int64_t>(nq, 48)) && aligned(codes, 16) && aligned(signs, 16);
   for (int64_t c0 = 0; c0 < n; c0 += L.chunk) {
     const int64_t cnt = std::min(L.chunk, n - c0);
-    st = v1_score(q, ytil, p, nq, nq, n, c0, cnt, codes, signs, norms, scores, L.chunk, 0, s);
+    if (tc) {
+      for (int64_t qb = 0; qb < nq; qb += 48) {  // query batches share one operand buffer
+        const int64_t nb = std::min<int64_t>(48, nq - qb);
+        st = tc_score(q, ytil + qb * q->d, p + qb * q->m, 1, nb, n, c0, cnt, codes, signs, norms,
+                      scores + qb * L.chunk, L.chunk, 0, reinterpret_cast<int8_t *>(ws + L.qop),
+                      reinterpret_cast<float4 *>(ws + L.qsc) + qb, s);
+        if (st != TQ_OK) return st;
+      }
+    } else {
+      st = v1_score(q, ytil, p, nq, nq, n, c0, cnt, codes, signs, norms, scores, L.chunk, 0, s);
+    }
     if (st != TQ_OK) return st;
     st = v1_topk_select(scores, nullptr, nq, L.chunk, cnt, kTopkSlice, c0, k, part_s + (c0 / kTopkSlice) * k,
                         part_i + (c0 / kTopkSlice) * k, L.nparts * k, s);

@@ -479,6 +479,21 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
     return st;
   }
 
+  {
+    // centroids as 16-bit fixed point split into two signed bytes (integer scorer)
+    double big = 0.0;
+    for (double c : q->centroids) big = std::max(big, std::fabs(c));
+    int e = 0;
+    std::frexp(big, &e);  // big < 2^e
+    q->score_cexp = 14 - e;  // |c| * 2^cexp < 2^14: the limbs stay within int8
+    const int L = 1 << q->w;
+    for (int k = 0; k < L; ++k) {
+      const long v = std::lrint(std::ldexp(q->centroids[k], q->score_cexp));
+      const long hi = (v + 128) >> 8;  // floor((v + 128) / 256)
+      q->score_ch[k] = (int8_t)hi;
+      q->score_cl[k] = (int8_t)(v - 256 * hi);
+    }
+  }
   KernelTables &kt = q->kt;
   kt.d = d;
   kt.w = q->w;

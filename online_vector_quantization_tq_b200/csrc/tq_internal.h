@@ -46,6 +46,9 @@ struct tq_quantizer {
   float tc_rho = 0.f;
   uint16_t *d_rot_bf16 = nullptr;  // Hadamard: d^1.5 R as two exact bf16 pieces [2][d][d]
   int *d_err = nullptr;          // device error word (bounded waits that timed out)
+  // integer scorer: centroid c_k ~ (256 * ch[k] + cl[k]) * 2^-score_cexp
+  int8_t score_ch[tq::kMaxLevels] = {}, score_cl[tq::kMaxLevels] = {};
+  int score_cexp = 0;
   tq::KernelTables kt{};
 };
 

@@ -219,3 +219,21 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 
 }  // namespace sm100
 }  // namespace tq
+
+namespace tq {
+namespace sm100 {
+// 1-D bulk copy global -> shared, completing on `bar` (16-byte aligned, size
+// a multiple of 16).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+}  // namespace sm100
+}  // namespace tq

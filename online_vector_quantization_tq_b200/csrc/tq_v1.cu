@@ -7,7 +7,7 @@
 //   k_gemm_nt       fp32 tiled C = A B^T with an element-wise epilogue; dense
 //                   (Haar) rotation, its QJL projection, dense query prep
 //   k_pack_rows     packs the dense path's per-coordinate codes and signs
-//   k_prep_fwht     queries: y~ = R y, p = S y~ for d in {32, 64, 128}
+//   k_prep_fwht_block  queries: y~ = R y, p = S y~ for d in {32, 64, 128}
 //   k_score_rows    asymmetric estimator, one thread per key, one query row
 //                   per grid row
 //   k_topk_*        per-block top-k of score rows, then a merge
@@ -225,34 +225,43 @@ __global__ void k_pack_rows(int d, int m, int64_t rows, const uint8_t *code, con
 }
 
 // ============================================================ queries
+// One block of D threads per query: sign flips and Walsh-Hadamard butterflies
+// in shared memory, then p = S y~ with each warp reducing whole rows of S.
 template <int D>
-__global__ void __launch_bounds__(128)
-k_prep_fwht(KernelTables kt, RowSource src, int64_t nq, float *ytil, float *p) {
-  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= nq) return;
-  float v[D];
-#pragma unroll
-  for (int j = 0; j < D; ++j) v[j] = src.at(row, j);
+__global__ void __launch_bounds__(D)
+k_prep_fwht_block(KernelTables kt, RowSource src, int64_t nq, float *ytil, float *p) {
+  __shared__ float v[D];
+  const int64_t row = blockIdx.x;
+  const int j = threadIdx.x;
+  float x = src.at(row, j);
 #pragma unroll
   for (int r = 0; r < 3; ++r) {
-    uint32_t words[D / 32];
+    const uint32_t word = kt.diag_bits[r * (D / 32) + j / 32];
+    x = ((word >> (j % 32)) & 1u) ? -x : x;
+    v[j] = x;
+    __syncthreads();
 #pragma unroll
-    for (int k = 0; k < D / 32; ++k) words[k] = kt.diag_bits[r * (D / 32) + k];
-    apply_signs<D>(v, words);
-    fwht_regs<D>(v);
+    for (int h = 1; h < D; h <<= 1) {
+      const float a = v[j], b = v[j ^ h];
+      x = (j & h) ? b - a : a + b;
+      __syncthreads();
+      v[j] = x;
+      __syncthreads();
+    }
   }
-  const float s = 1.0f / (float(D) * sqrtf(float(D)));
-#pragma unroll
-  for (int j = 0; j < D; ++j) {
-    v[j] *= s;
-    ytil[row * D + j] = v[j];
-  }
-  for (int i = 0; i < D; ++i) {
+  x *= 1.0f / (float(D) * sqrtf(float(D)));
+  v[j] = x;
+  ytil[row * D + j] = x;
+  __syncthreads();
+  const int lane = j % 32, warp = j / 32;
+  for (int i = warp; i < D; i += D / 32) {
     const float *srow = kt.qjl32 + (size_t)i * D;
-    float z = 0.f;
+    float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < D; ++j) z = fmaf(srow[j], v[j], z);
-    p[row * D + i] = z;
+    for (int k = lane; k < D; k += 32) acc = fmaf(srow[k], v[k], acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) p[row * D + i] = acc;
   }
 }
 
@@ -501,9 +510,9 @@ tq_status v1_prepare_queries(const tq_quantizer *q, const RowSource &src, int64_
   const int d = q->d;
   if (q->rotation == TQ_ROT_HADAMARD && (d == 32 || d == 64 || d == 128)) {
     switch (d) {
-      case 32: k_prep_fwht<32><<<ceil_div_i(nq, 128), 128, 0, st>>>(q->kt, src, nq, ytil, p); break;
-      case 64: k_prep_fwht<64><<<ceil_div_i(nq, 128), 128, 0, st>>>(q->kt, src, nq, ytil, p); break;
-      case 128: k_prep_fwht<128><<<ceil_div_i(nq, 128), 128, 0, st>>>(q->kt, src, nq, ytil, p); break;
+      case 32: k_prep_fwht_block<32><<<(unsigned)nq, 32, 0, st>>>(q->kt, src, nq, ytil, p); break;
+      case 64: k_prep_fwht_block<64><<<(unsigned)nq, 64, 0, st>>>(q->kt, src, nq, ytil, p); break;
+      case 128: k_prep_fwht_block<128><<<(unsigned)nq, 128, 0, st>>>(q->kt, src, nq, ytil, p); break;
     }
     TQ_CHECK_LAUNCH();
     return TQ_OK;
