@@ -66,7 +66,8 @@ typedef enum {
   TQ_ERR_ALIGNMENT = 3,    /* a pointer or leading dimension breaks the stated alignment */
   TQ_ERR_NOMEM = 4,        /* host or device allocation of the quantizer tables failed */
   TQ_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed        */
-  TQ_ERR_WORKSPACE = 6     /* workspace pointer null or smaller than required    */
+  TQ_ERR_WORKSPACE = 6,    /* workspace pointer null or smaller than required    */
+  TQ_ERR_TOO_LARGE = 7     /* request needs more than a fixed internal buffer    */
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
@@ -188,6 +189,36 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups,
                    const void *codes, const void *signs, const float *norms,
                    int64_t keys_per_group, float *out, int accumulate,
                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------- score, no allocation
+ * tq_score_noalloc: the same scores as tq_score, for callers that cannot hand
+ * the library a workspace.  (No counterpart in the TurboQuant pages; this is
+ * an interface for embedding.)  Typical such callers: code running while a
+ * framework's caching allocator holds the device memory (a direct allocation
+ * would fail or fragment that pool), latency-critical paths where the device
+ * synchronization an allocation can cause is not acceptable, and plugin hosts
+ * that forbid device allocation once started.
+ *
+ * Scratch comes from one buffer of TQ_NOALLOC_SCRATCH_BYTES compiled into the
+ * library as a device variable: every GPU that loads the library holds it
+ * until the process exits.  Arguments, layouts and results are exactly those
+ * of tq_score.  The call allocates and frees nothing.
+ *   - Needed scratch: per query 4*(d + m) + 16 bytes, plus 384 bytes for each
+ *     of roundup(5*G, 16) operand rows per group when G <= 48 (each piece
+ *     rounded up to 256 bytes).  Larger requests return TQ_ERR_TOO_LARGE
+ *     before anything is launched.
+ *   - The first call on each device looks up the buffer's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     outside any stream capture.
+ *   - All calls share the one buffer and it keeps the last call's contents:
+ *     calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on it and return wrong scores.  Order them on one stream. */
+#define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+tq_status tq_score_noalloc(const tq_quantizer *q, const float *y, int64_t groups,
+                           int64_t G, int64_t ldy, const int32_t *ychan,
+                           const void *codes, const void *signs,
+                           const float *norms, int64_t keys_per_group,
+                           float *out, int accumulate, void *stream);
 
 /* ---------------------------------------------------------------- top-k
  * tq_topk: the k highest estimates per query over n keys (TurboQuant article

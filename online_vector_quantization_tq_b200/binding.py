@@ -20,7 +20,8 @@ TQ_F32, TQ_BF16 = 0, 1
 ROTATIONS = {"auto": 0, "hadamard": 1, "haar": 2}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration",
           3: "misaligned pointer or leading dimension", 4: "out of memory",
-          5: "CUDA error", 6: "workspace missing or too small"}
+          5: "CUDA error", 6: "workspace missing or too small",
+          7: "request exceeds the fixed internal scratch buffer"}
 
 _lib = None
 
@@ -64,6 +65,7 @@ def lib() -> ctypes.CDLL:
         "tq_score": (i32, [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp, i32, vp, sz, vp]),
         "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
         "tq_topk": (i32, [vp, vp, i64, i64, vp, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
+        "tq_score_noalloc": (i32, [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp, i32, vp]),
         "tq_outlier_workspace_bytes": (sz, [i64, i32]),
         "tq_outlier_channels": (i32, [vp, i32, i64, i64, i32, i64, i32, vp, vp, vp, sz, vp]),
     }

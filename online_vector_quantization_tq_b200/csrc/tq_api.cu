@@ -4,6 +4,7 @@
 // contract of each call.
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "tq_kernels.h"
@@ -317,3 +318,71 @@ tq_status tq_outlier_channels(const void *x, tq_dtype dtype, int64_t groups, int
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation scoring
+// Scratch of tq_score_noalloc: a fixed device buffer, so the call needs no
+// workspace from the caller and allocates nothing.  Host code cannot use the
+// symbol itself as a device pointer; its address is looked up once per
+// device (with that device current) and passed to the kernels.
+static __device__ __align__(256) unsigned char g_tq_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 64;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+tq_status noalloc_scratch(int dev, void **out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (dev < 0 || dev >= kMaxDevices) return TQ_ERR_UNSUPPORTED;
+  if (!g_noalloc_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_tq_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return TQ_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return TQ_OK;
+}
+}  // namespace
+
+extern "C" tq_status tq_score_noalloc(const tq_quantizer *q, const float *y, int64_t groups, int64_t G,
+                                      int64_t ldy, const int32_t *ychan, const void *codes, const void *signs,
+                                      const float *norms, int64_t keys_per_group, float *out, int accumulate,
+                                      void *stream) {
+  if (!q || groups < 0 || G < 0 || keys_per_group < 0) return TQ_ERR_INVALID_ARG;
+  const int64_t nq = groups * G;
+  bool empty = false;
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, G > 0 ? G : 1, &empty);
+  if (st != TQ_OK || empty) return st;
+  if (!codes || !signs || !norms || !out) return TQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out, 4)) return TQ_ERR_ALIGNMENT;
+  if (keys_per_group == 0) return TQ_OK;
+  const bool tc = tc_score_supported(q, G) && aligned(codes, 16) && aligned(signs, 16);
+  // scratch pieces for this call: y~, p, then (integer scorer only) its
+  // query operand and per-query scales
+  const size_t b_ytil = round_up((size_t)nq * q->d * 4, 256);
+  const size_t b_p = round_up((size_t)nq * q->m * 4, 256);
+  const size_t b_qop = tc ? round_up(tc_score_qop_bytes(q, groups, G), 256) : 0;
+  const size_t b_qsc = tc ? round_up((size_t)nq * 16, 256) : 0;
+  if (b_ytil + b_p + b_qop + b_qsc > TQ_NOALLOC_SCRATCH_BYTES) return TQ_ERR_TOO_LARGE;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  void *base = nullptr;
+  st = noalloc_scratch(q->device, &base);
+  if (st != TQ_OK) return st;
+  char *ws = static_cast<char *>(base);
+  float *ytil = reinterpret_cast<float *>(ws);
+  float *p = reinterpret_cast<float *>(ws + b_ytil);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RowSource src{y, ldy, ychan, G, q->d, 0};
+  st = v1_prepare_queries(q, src, nq, ytil, p, s);
+  if (st != TQ_OK) return st;
+  if (tc)  // the operand region is cleared inside tc_score before it is filled
+    return tc_score(q, ytil, p, groups, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
+                    keys_per_group, accumulate, reinterpret_cast<int8_t *>(ws + b_ytil + b_p),
+                    reinterpret_cast<float4 *>(ws + b_ytil + b_p + b_qop), s);
+  return v1_score(q, ytil, p, nq, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
+                  keys_per_group, accumulate, s);
+}

@@ -315,6 +315,7 @@ const char *tq_status_string(tq_status s) {
     case TQ_ERR_NOMEM: return "out of memory";
     case TQ_ERR_CUDA: return "CUDA error";
     case TQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case TQ_ERR_TOO_LARGE: return "request exceeds the fixed internal scratch buffer";
   }
   return "unknown status";
 }
