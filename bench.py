@@ -7,7 +7,10 @@ step per second, summed over ranks (weak scaling: every rank runs its own
 layer; the path shards by key with no collective).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
-                  [--workload kv|tiny|decode]
+                  [--workload kv|tiny|kv_mixed|decode|ann] [--queries Q]
+
+The default (kv) is the headline line; the other workloads print a line with
+per-phase times on one GPU.
 
 Rank 0 prints one JSON line.  Timing: CUDA events on the launching stream,
 barrier + synchronize around the K timed steps, max over ranks.  The keys
@@ -45,23 +48,28 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    """nvidia-smi samples of SM clock and throttle reasons during a region.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    Samples every GPU the driver shows and keeps the one whose UUID matches
+    the CUDA device (or the only one, when just one is visible)."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
+    def __init__(self, uuid: str):
+        self.uuid = (uuid or "").lower().replace("gpu-", "")
         self.proc = None
         self.out = None
+        self.error = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        except Exception as e:  # no nvidia-smi
+            self.error = str(e)
             self.proc = None
         return self
 
@@ -69,30 +77,35 @@ class ClockSampler:
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.out, err = self.proc.communicate(timeout=5)
+                if not self.out:
+                    self.error = (err or "").strip()[:200]
             except Exception:
                 self.proc.kill()
                 self.out = ""
 
     def summary(self):
-        if not self.out:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
+        lines = [[x.strip() for x in ln.split(",")] for ln in (self.out or "").strip().splitlines()]
+        lines = [ln for ln in lines if len(ln) >= 8]
+        uuids = sorted({ln[0].lower().replace("gpu-", "") for ln in lines})
+        if self.uuid in uuids:
+            lines = [ln for ln in lines if ln[0].lower().replace("gpu-", "") == self.uuid]
+        elif len(uuids) > 1:
+            lines = [ln for ln in lines if ln[0].lower().replace("gpu-", "") == uuids[0]]
+        sm, mx, reasons = [], None, set()
+        for ln in lines:
             try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
+                sm.append(float(ln[1]))
+                mx = float(ln[2])
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[3:7]):
+            for nm, v in zip(names, ln[4:8]):
                 if v.lower() == "active":
                     reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "error": self.error}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm), "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------------------- workloads
@@ -140,16 +153,26 @@ def run_tq(args, rank, world, local):
             c.record(stream)
             record.append((a, b_, c))
 
+    w0 = torch.cuda.Event(enable_timing=True)
+    w1 = torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
     for _ in range(args.warmup):
         step()
+    w1.record(stream)
     torch.cuda.synchronize(dev)
+    warm_ms = w0.elapsed_time(w1) / max(1, args.warmup)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     props = torch.cuda.get_device_properties(dev)
-    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
     recs = []
-    with ClockSampler(gpu_id) as clk:
+    with ClockSampler(str(getattr(props, "uuid", ""))) as clk:
+        # keep the GPU busy for ~1 s before the timed steps so the clock
+        # samples (every 100 ms) cover the load
+        pre = max(1, int(1.0 / max(warm_ms * 1e-3, 1e-5)))
+        for _ in range(pre):
+            step()
+        torch.cuda.synchronize(dev)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -245,8 +268,133 @@ def run_tq(args, rank, world, local):
         dist.destroy_process_group()
 
 
-# kernels of libtq launched per step: encode (1), query preparation (1), scoring (1)
-LAUNCHES_PER_STEP = 3
+def run_workload(args):
+    """The other workloads on one GPU (tiny, kv_mixed, decode, ann).  Prints
+    one JSON line with the step time, per-phase times and algorithmic GB/s."""
+    import torch
+
+    import online_vector_quantization_tq_b200 as tq
+    import workloads as wl
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    phases = {}
+
+    def timed(name, fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        phases.setdefault(name, []).append((a, b))
+
+    if args.workload == "tiny":
+        x = torch.from_numpy(wl.tiny_keys()).to(dev)
+        y = torch.from_numpy(wl.tiny_queries()).to(dev)
+        q = tq.tq_codebook(128, 3, seed=0)
+        enc = q.empty_encoded(x.shape[0], dev)
+        ws = tq.topk_workspace(q, y.shape[0], x.shape[0], 10, dev)
+        n_units, unit = x.shape[0], "keys/s"
+        bytes_ = {"encode": x.shape[0] * (512 + q.code_bytes + q.sign_bytes + 8),
+                  "topk": x.shape[0] * (q.code_bytes + q.sign_bytes + 8)}
+        desc = "tiny: 4096 keys d=128 fp32 N(0,1), b=3, 16 queries, top-10"
+
+        def step():
+            timed("encode", lambda: tq.tq_encode(q, x, out=enc, stream=stream))
+            timed("topk", lambda: tq.tq_topk(q, y, enc, 10, workspace=ws, stream=stream))
+    elif args.workload == "kv_mixed":
+        kpg, groups, G = 131072, 8, 4
+        xs = np.stack([wl.kv_head_keys(h, kpg) for h in range(groups)]).reshape(-1, 128)
+        x = torch.from_numpy(xs).to(dev).to(torch.bfloat16)
+        y = torch.from_numpy(wl.kv_queries()).to(dev)
+        sel, rest = tq.tq_outlier_channels(x, groups, kpg, 32)
+        qa, qb = tq.tq_codebook(32, 5, seed=0), tq.tq_codebook(96, 3, seed=0)
+        ea, eb = qa.empty_encoded(x.shape[0], dev), qb.empty_encoded(x.shape[0], dev)
+        out = torch.empty((groups * G, kpg), device=dev)
+        wsa, wsb = tq.score_workspace(qa, groups * G, dev), tq.score_workspace(qb, groups * G, dev)
+        n_units, unit = x.shape[0], "keys/s"
+        bytes_ = {"encode": x.shape[0] * (256 + 72), "score": x.shape[0] * (72 + 16)}
+        desc = ("kv_mixed: kv tensors, per head 32 highest-RMS channels at b=5 (d=32) + 96 at b=3 (d=96, Haar), "
+                "scores summed")
+
+        def step():
+            timed("encode", lambda: (tq.tq_encode(qa, x, out=ea, chan=sel, chan_rows=kpg, stream=stream),
+                                     tq.tq_encode(qb, x, out=eb, chan=rest, chan_rows=kpg, stream=stream)))
+            timed("score", lambda: (tq.tq_score(qa, y, groups, G, ea, kpg, out=out, ychan=sel, workspace=wsa,
+                                                stream=stream),
+                                    tq.tq_score(qb, y, groups, G, eb, kpg, out=out, accumulate=True, ychan=rest,
+                                                workspace=wsb, stream=stream)))
+    elif args.workload == "decode":
+        groups, kpg, G = 256, 32768, 4
+        q = tq.tq_codebook(128, 3, seed=0)
+        cache = q.empty_encoded(groups * kpg, dev)
+        for g in range(groups):
+            xg = torch.from_numpy(wl.decode_group_keys(g, kpg)).to(dev).to(torch.bfloat16)
+            tq.tq_encode(q, xg, out=tq.binding.Encoded(cache.codes[g * kpg:], cache.signs[g * kpg:],
+                                                        cache.norms[g * kpg:]))
+            if g == 0:
+                new = torch.empty((groups, 128), dtype=torch.bfloat16, device=dev)
+            new[g] = xg[kpg - 1]
+        tail = tq.binding.Encoded(cache.codes[kpg - 1:], cache.signs[kpg - 1:], cache.norms[kpg - 1:])
+        y = torch.from_numpy(wl.decode_queries(groups)).to(dev)
+        out = torch.empty((groups * G, kpg), device=dev)
+        ws = tq.score_workspace(q, groups * G, dev)
+        n_units, unit = groups * kpg, "keys/s"
+        bytes_ = {"append": groups * (256 + 56), "score": groups * kpg * (56 + 16)}
+        desc = "decode: 256 caches x 32768 keys, d=128, b=3; step = append 256 keys + score 4 heads per cache"
+
+        def step():
+            timed("append", lambda: tq.tq_encode(q, new, out=tail, out_stride=kpg, stream=stream))
+            timed("score", lambda: tq.tq_score(q, y, groups, G, cache, kpg, out=out, workspace=ws, stream=stream))
+    elif args.workload == "ann":
+        n, d, nq = 1_000_000, 1536, args.queries
+        x = torch.empty((n, d), device=dev)
+        for c in range((n + wl.ANN_CHUNK - 1) // wl.ANN_CHUNK):
+            blk = wl.ann_chunk(c, n, d)
+            x[c * wl.ANN_CHUNK:c * wl.ANN_CHUNK + blk.shape[0]] = torch.from_numpy(blk).to(dev)
+        y = torch.from_numpy(wl.ann_queries(1024, d)[:nq]).to(dev)
+        q = tq.tq_codebook(d, 4, seed=0)
+        enc = q.empty_encoded(n, dev)
+        wse = torch.empty(max(1, tq.lib().tq_encode_workspace_bytes(q.handle, n)), dtype=torch.uint8, device=dev)
+        ws = tq.topk_workspace(q, nq, n, 10, dev)
+        n_units, unit = n, "vectors/s"
+        bytes_ = {"encode": n * (4 * d + q.code_bytes + q.sign_bytes + 8),
+                  "topk": n * (q.code_bytes + q.sign_bytes + 8)}
+        desc = f"ann: 1e6 x 1536 fp32 (std i^-0.5, L2-normalised), Haar, b=4; {nq} queries, top-10"
+
+        def step():
+            timed("encode", lambda: tq.tq_encode(q, x, out=enc, workspace=wse, stream=stream))
+            timed("topk", lambda: tq.tq_topk(q, y, enc, 10, workspace=ws, stream=stream))
+    else:
+        raise SystemExit(f"unknown workload {args.workload}")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    phases.clear()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / args.steps
+    peak, peak_kind = _peaks()
+    ph = {}
+    for name, evs in phases.items():
+        pm = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        gbs = bytes_[name] / (pm * 1e-3) / 1e9
+        ph[name] = {"ms": pm, "algorithmic_GBps": gbs, "frac_of_measured_hbm": gbs / peak}
+    line = {"metric": METRIC, "value": n_units / (ms * 1e-3), "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "data": "synthetic", "config": {"workload": desc}, "phases": ph,
+            "peak_hbm_GBps": peak, "peak_kind": peak_kind}
+    print(json.dumps(line), flush=True)
+
+
+# kernels of libtq launched per step: encode (1), query preparation (1), query
+# operand of the integer scorer (1, plus one memset of it), scoring (1)
+LAUNCHES_PER_STEP = 4
 
 
 def _oracle_sample(n_keys):
@@ -307,15 +455,21 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", choices=["kv", "tiny", "kv_mixed", "decode", "ann"], default="kv")
+    ap.add_argument("--queries", type=int, default=16, help="ann workload: number of queries")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.workload != "kv":
+        if rank == 0:
+            run_workload(args)
         return
     run_tq(args, rank, world, local)
 

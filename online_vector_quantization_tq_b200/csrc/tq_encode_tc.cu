@@ -115,7 +115,6 @@ k_encode_tc(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   const int row = tid & (kRows - 1);
   const int half = tid >> 7;
   const int c0 = half ? SPL : 0;
-  const int c1 = half ? D : SPL;
   constexpr int NC0 = SPL, NC1 = D - SPL;
   const int nc = half ? NC1 : NC0;
   const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
@@ -351,7 +350,7 @@ k_encode_tc(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
 
   // ---- drain: sign bits of the last tile
   if (!failed && it > 0) {
-    const bool ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 4);
+    const bool ok = __syncthreads_and(sm100::mbar_wait(&bars[3], ph_qjl, p.err, 4)) != 0;  // CTA-uniform
     sm100::tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -594,6 +593,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   const uint32_t idesc_rot = sm100::idesc_bf16_f32(kRows, D);
   const uint32_t idesc_qjl = sm100::idesc_f16_f32(kRows, D);
   const int first = blockIdx.x, stride = gridDim.x;
+  const int nloc = first < p.ntiles ? (p.ntiles - first + stride - 1) / stride : 0;
 
   auto issue_rot = [&](int buf, uint32_t ucol) {
     const uint32_t xa = sm100::smem_u32(sX + buf * SM::kXBytes), br = sm100::smem_u32(sBr);
@@ -607,137 +607,174 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       }
     sm100::mma_commit(&bars[2]);
   };
+  auto issue_qjl = [&]() {
+    const uint32_t ar = sm100::smem_u32(sAr), bs = sm100::smem_u32(sBs);
+#pragma unroll
+    for (int ks = 0; ks < 2 * D / 16; ++ks) {
+      const int kk = ks % (D / 16);
+      const uint64_t a = sm100::desc_sw64(ar + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+      const uint64_t b = sm100::desc_sw64(bs + (kk >> 1) * (D * 64) + (kk & 1) * 32);
+      sm100::mma_f16(tmem + kColZ, a, b, idesc_qjl, ks != 0);
+    }
+    sm100::mma_commit(&bars[3]);
+  };
   auto issue_tma = [&](int buf, int tile) {
     sm100::mbar_expect_tx(&bars[buf], SM::kXBytes);
 #pragma unroll
     for (int bx = 0; bx < NB; ++bx)
       sm100::tma_load_2d(sX + buf * SM::kXBytes + bx * (kRows * 128), &xmap, bx * 64, tile * kRows, &bars[buf]);
   };
+  // Per-row partial sums live in TMEM columns, double-buffered by tile
+  // parity: ||U||^2 parts at kColScr + 16*par + pc, gamma^2 parts at +8.
+  auto norm_col = [&](int par) { return (uint32_t)(kColScr + 16 * par); };
+  auto gam_col = [&](int par) { return (uint32_t)(kColScr + 16 * par + 8); };
+  auto row_partial = [&](uint32_t ucol, uint32_t scol) {
+    uint32_t u[32];
+    sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, u);
+    sm100::tmem_wait_ld();
+    float2 ss = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float2 v = make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1]));
+      ss = __ffma2_rn(v, v, ss);
+    }
+    sm100::tmem_st1(tmem + lane + scol + pc, __float_as_uint(ss.x + ss.y));
+  };
+  auto sum_parts = [&](uint32_t scol) {
+    uint32_t parts[4];
+    sm100::tmem_ld4(tmem + lane + scol, parts);
+    sm100::tmem_wait_ld();
+    float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < P; ++k) v += __uint_as_float(parts[k]);
+    return v;
+  };
+  auto sign_word = [&]() {
+    uint32_t z[32];
+    sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+    sm100::tmem_wait_ld();
+    uint32_t wbits = 0u;
+#pragma unroll
+    for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+    return ~wbits;
+  };
 
-  // thread 0's bookkeeping of asynchronous work in flight
+  // thread 0's bookkeeping of loads in flight
   bool pend_full[2] = {false, false};
   uint32_t ph_full[2] = {0u, 0u};
-  bool failed = false;
-  if (tid == 0 && first < p.ntiles) {
-    issue_tma(0, first);
-    pend_full[0] = true;
-    if (first + stride < p.ntiles) {
-      issue_tma(1, first + stride);
-      pend_full[1] = true;
-    }
-    if (!sm100::mbar_wait(&bars[0], ph_full[0], p.err, 11)) failed = true;
-    ph_full[0] ^= 1u;
-    pend_full[0] = false;
-    sm100::tc_fence_after();
-    if (!failed) issue_rot(0, kColU0);
-  }
-
   uint32_t ph_rot = 0u, ph_qjl = 0u;
-  float prev_norm = 0.f, prev_gamma = 0.f;
-  int64_t prev_row = -1;
-  int it = 0;
-  for (int t = first; t < p.ntiles; t += stride, ++it) {
-    const int buf = it & 1;
-    const int64_t grow = (int64_t)t * kRows + row;
-    const uint32_t ucol = (it & 1) ? 128u : 0u;
-    // ---- (1) rotated tile -> registers, ||U||^2 partial -> TMEM scratch
+  bool failed = false;
+
+  // ---- prologue: tiles 0 and 1 loaded, rotation of tile 0, its norm parts
+  if (nloc > 0) {
+    if (tid == 0) {
+      issue_tma(0, first);
+      pend_full[0] = true;
+      if (nloc > 1) {
+        issue_tma(1, first + stride);
+        pend_full[1] = true;
+      }
+      failed = !sm100::mbar_wait(&bars[0], ph_full[0], p.err, 11);
+      ph_full[0] ^= 1u;
+      pend_full[0] = false;
+      sm100::tc_fence_after();
+      if (!failed) issue_rot(0, kColU0);
+    }
     bool ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 12);
     ph_rot ^= 1u;
     sm100::tc_fence_after();
+    row_partial(kColU0, norm_col(0));
+    sm100::tmem_wait_st();
+    sm100::tc_fence_before();
+    failed = __syncthreads_or(!ok || failed) != 0;
+    sm100::tc_fence_after();
+    if (tid == 0 && !failed) {
+      if (nloc > 2) {
+        issue_tma(0, first + 2 * stride);  // tile 0's rotation is done with buffer 0
+        pend_full[0] = true;
+      }
+      if (nloc > 1) {
+        failed = !sm100::mbar_wait(&bars[1], ph_full[1], p.err, 13);
+        ph_full[1] ^= 1u;
+        pend_full[1] = false;
+        sm100::tc_fence_after();
+        if (!failed) issue_rot(1, 128u);
+      }
+    }
+  }
+
+  float prev_norm = 0.f;
+  int64_t prev_row = -1;
+  const float2 big2 = make_float2(kBig, kBig);
+  const float2 half2v = make_float2(0.5f, 0.5f);
+  const float2 base2 = make_float2(8388608.0f + (float)(HALF - 1), 8388608.0f + (float)(HALF - 1));
+  int it = 0;
+  for (; it < nloc && !failed; ++it) {
+    const int t = first + it * stride;
+    const int par = it & 1;
+    const uint32_t ucol = par ? 128u : 0u;
+    const int64_t grow = (int64_t)t * kRows + row;
+    bool ok = true;
+    // ---- (a) this tile's rotated row (its MMA completed before the last barrier)
+    const float nacc = sqrtf(sum_parts(norm_col(par)));
+    const float nrm = nacc * p.rho;
+    const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;  // zero rows: u = -0 -> lower middle code
+    const float2 sv2 = make_float2(s_v, s_v);
     uint32_t acc[32];
     sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
     sm100::tmem_wait_ld();
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) ss = fmaf(__uint_as_float(acc[j]), __uint_as_float(acc[j]), ss);
-    sm100::tmem_st1(tmem + lane + kColScr + pc, __float_as_uint(ss));
-    sm100::tmem_wait_st();
-    sm100::tc_fence_before();
-    failed |= __syncthreads_or(!ok || failed) != 0;
-    if (failed) break;
-    sm100::tc_fence_after();
-    if (tid == 0) {
-      // x tile t has been consumed: refill this buffer, start the next rotation
-      const int t2 = t + 2 * stride;
-      if (t2 < p.ntiles) {
-        issue_tma(buf, t2);
-        pend_full[buf] = true;
-      }
-      const int t1 = t + stride;
-      if (t1 < p.ntiles) {
-        const int b1 = buf ^ 1;
-        if (!sm100::mbar_wait(&bars[b1], ph_full[b1], p.err, 13)) failed = true;
-        ph_full[b1] ^= 1u;
-        pend_full[b1] = false;
-        sm100::tc_fence_after();
-        if (!failed) issue_rot(b1, ucol ^ 128u);
-      }
-    }
-    // ---- (3a) norm, codes, residual split (kept in registers)
-    uint32_t parts[4];
-    sm100::tmem_ld4(tmem + lane + kColScr, parts);
-    sm100::tmem_wait_ld();
-    float nacc = 0.f;
-#pragma unroll
-    for (int k = 0; k < P; ++k) nacc += __uint_as_float(parts[k]);
-    nacc = sqrtf(nacc);
-    const float nrm = nacc * p.rho;
-    const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;  // zero rows: u = -0 -> lower middle code
     uint32_t cw[W];
 #pragma unroll
     for (int k = 0; k < W; ++k) cw[k] = 0u;
     uint32_t hi[16], lo[16];
-    float g2 = 0.f;
+    float2 g2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
-      float rr[2];
+      const float2 us = __fmul2_rn(make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])), sv2);
+      const float2 usb = __fmul2_rn(us, big2);
+      float2 cm = make_float2(dC[0], dC[0]), m = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float us = __uint_as_float(acc[j + e]) * s_v;
-        const float usb = us * kBig;
-        float cm = dC[0], m = 0.f;
-#pragma unroll
-        for (int k = 1; k < HALF; ++k) {
-          const float st = __saturatef(__fmaf_rn(us, usb, nT2B[k]));
-          cm = __fmaf_rn(st, dC[k], cm);
-          m += st;
-        }
-        // s = +-1 from the sign bit (u = -0 takes the lower middle code)
-        const float sg = __uint_as_float((__float_as_uint(us) & 0x80000000u) | 0x3F800000u);
-        const float s01 = __fmaf_rn(sg, 0.5f, 0.5f);
-        // code = HALF-1+s01 + s*m, as the low bits of 2^23 + code
-        const float codef = __fmaf_rn(sg, m, s01 + (8388608.0f + (float)(HALF - 1)));
-        rr[e] = __fmaf_rn(-sg, cm, us);
-        pack_code<W>(cw, j + e, __float_as_uint(codef) & (uint32_t)(L - 1));
-        g2 = fmaf(rr[e], rr[e], g2);
+      for (int k = 1; k < HALF; ++k) {
+        const float2 st = make_float2(__saturatef(__fmaf_rn(us.x, usb.x, nT2B[k])),
+                                      __saturatef(__fmaf_rn(us.y, usb.y, nT2B[k])));
+        cm = __ffma2_rn(st, make_float2(dC[k], dC[k]), cm);
+        m = __fadd2_rn(m, st);
       }
-      const __half2 h = __floats2half2_rn(rr[0], rr[1]);
+      // s = +-1 from the sign bit (u = -0 takes the lower middle code)
+      const uint32_t bx = __float_as_uint(us.x) & 0x80000000u, by = __float_as_uint(us.y) & 0x80000000u;
+      const float2 sg = make_float2(__uint_as_float(bx | 0x3F800000u), __uint_as_float(by | 0x3F800000u));
+      const float2 nsg = make_float2(__uint_as_float(bx ^ 0xBF800000u), __uint_as_float(by ^ 0xBF800000u));
+      const float2 cb = __fadd2_rn(__ffma2_rn(sg, half2v, half2v), base2);
+      const float2 codef = __ffma2_rn(sg, m, cb);  // 2^23 + code
+      const float2 rr = __ffma2_rn(nsg, cm, us);   // u - c[code]
+      pack_code<W>(cw, j, __float_as_uint(codef.x) & (uint32_t)(L - 1));
+      pack_code<W>(cw, j + 1, __float_as_uint(codef.y) & (uint32_t)(L - 1));
+      g2 = __ffma2_rn(rr, rr, g2);
+      const __half2 h = __floats2half2_rn(rr.x, rr.y);
       const float2 hf = __half22float2(h);
       hi[j / 2] = *reinterpret_cast<const uint32_t *>(&h);
-      lo[j / 2] = pack_half2(rr[0] - hf.x, rr[1] - hf.y);
+      const float2 lf = __fadd2_rn(rr, make_float2(-hf.x, -hf.y));
+      lo[j / 2] = pack_half2(lf.x, lf.y);
     }
     if (grow < p.n) {
       uint32_t *dst = p.codes + grow * p.out_stride * (W * D / 32) + pc * W;
 #pragma unroll
       for (int k = 0; k < W; ++k) dst[k] = cw[k];
     }
-    // ---- (2) sign bits of the previous tile
+    // ---- (b) sign bits and norms of the previous tile
     if (it > 0) {
-      ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 14) && ok;
+      ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 14);
       ph_qjl ^= 1u;
       sm100::tc_fence_after();
-      uint32_t z[32];
-      sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
-      sm100::tmem_wait_ld();
-      uint32_t wbits = 0u;
-#pragma unroll
-      for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+      // TMEM loads are warp-collective: every lane runs them, only stores are guarded
+      const uint32_t sw = sign_word();
+      const float gam = pc == 0 ? sqrtf(sum_parts(gam_col(par ^ 1))) * (1.0f / kRScale) : 0.f;
       if (prev_row >= 0 && prev_row < p.n) {
-        p.signs[prev_row * p.out_stride * (D / 32) + pc] = ~wbits;
-        if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, prev_gamma);
+        p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
+        if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
       }
     }
-    // ---- (3b) residual operand, gamma^2 partial
+    // ---- (c) residual operand
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       *reinterpret_cast<uint4 *>(sAr + pc * (kRows * 64) + sm100::sw64_offset(row, k)) =
@@ -745,51 +782,49 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       *reinterpret_cast<uint4 *>(sAr + (P + pc) * (kRows * 64) + sm100::sw64_offset(row, k)) =
           make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
     }
-    sm100::tmem_st1(tmem + lane + kColScr + 4 + pc, __float_as_uint(g2));
+    // ---- (d) norm parts of the next tile, gamma parts of this one
+    if (it + 1 < nloc) {
+      ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 15) && ok;
+      ph_rot ^= 1u;
+      sm100::tc_fence_after();
+      row_partial(ucol ^ 128u, norm_col(par ^ 1));
+    }
+    sm100::tmem_st1(tmem + lane + gam_col(par) + pc, __float_as_uint(g2.x + g2.y));
     sm100::tmem_wait_st();
     sm100::fence_proxy_async();
     sm100::tc_fence_before();
-    failed |= __syncthreads_or(!ok || failed) != 0;
+    failed = __syncthreads_or(!ok || failed) != 0;
     if (failed) break;
     sm100::tc_fence_after();
-    // ---- (4) QJL projection of this tile
+    // ---- (e) QJL projection of this tile; the rotation two tiles ahead
     if (tid == 0) {
-      const uint32_t ar = sm100::smem_u32(sAr), bs = sm100::smem_u32(sBs);
-#pragma unroll
-      for (int ks = 0; ks < 2 * D / 16; ++ks) {
-        const int kk = ks % (D / 16);
-        const uint64_t a = sm100::desc_sw64(ar + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
-        const uint64_t b = sm100::desc_sw64(bs + (kk >> 1) * (D * 64) + (kk & 1) * 32);
-        sm100::mma_f16(tmem + kColZ, a, b, idesc_qjl, ks != 0);
+      issue_qjl();
+      if (it + 3 < nloc) {  // tile it+1's rotation is done with its buffer
+        issue_tma(par ^ 1, first + (it + 3) * stride);
+        pend_full[par ^ 1] = true;
       }
-      sm100::mma_commit(&bars[3]);
-    }
-    float gsum = 0.f;
-    if (pc == 0) {
-      sm100::tmem_ld4(tmem + lane + kColScr + 4, parts);
-      sm100::tmem_wait_ld();
-#pragma unroll
-      for (int k = 0; k < P; ++k) gsum += __uint_as_float(parts[k]);
+      if (it + 2 < nloc) {
+        failed = !sm100::mbar_wait(&bars[par], ph_full[par], p.err, 17);
+        ph_full[par] ^= 1u;
+        pend_full[par] = false;
+        sm100::tc_fence_after();
+        if (!failed) issue_rot(par, ucol);  // U of this tile has been read
+      }
     }
     prev_norm = nrm;
-    prev_gamma = sqrtf(gsum) * (1.0f / kRScale);
     prev_row = grow;
   }
 
-  // ---- drain: sign bits of the last tile
+  // ---- drain: sign bits and norms of the last tile
   if (!failed && it > 0) {
-    const bool ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 15);
+    const bool ok = __syncthreads_and(sm100::mbar_wait(&bars[3], ph_qjl, p.err, 18)) != 0;  // CTA-uniform
     sm100::tc_fence_after();
     if (ok) {
-      uint32_t z[32];
-      sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
-      sm100::tmem_wait_ld();
-      uint32_t wbits = 0u;
-#pragma unroll
-      for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+      const uint32_t sw = sign_word();
+      const float gam = pc == 0 ? sqrtf(sum_parts(gam_col((it - 1) & 1))) * (1.0f / kRScale) : 0.f;
       if (prev_row >= 0 && prev_row < p.n) {
-        p.signs[prev_row * p.out_stride * (D / 32) + pc] = ~wbits;
-        if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, prev_gamma);
+        p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
+        if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
       }
     }
   }

@@ -262,6 +262,8 @@ void free_device(tq_quantizer *q) {
   cudaFree(q->d_rot);
   cudaFree(q->d_qjl16);
   cudaFree(q->d_qjl32);
+  cudaFree(q->d_qjl32t);
+  q->d_qjl32t = nullptr;
   q->d_diag_bits = nullptr;
   q->d_rot = nullptr;
   q->d_qjl16 = nullptr;
@@ -410,6 +412,12 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
   if (st == TQ_OK) st = upload(&q->d_qjl16, q->qjl16.data(), q->qjl16.size());
   if (st == TQ_OK) st = upload(&q->d_qjl32, s32.data(), s32.size());
   if (st == TQ_OK) {
+    std::vector<float> st32((size_t)m * d);
+    for (int i = 0; i < m; ++i)
+      for (int j = 0; j < d; ++j) st32[(size_t)j * m + i] = s32[(size_t)i * d + j];
+    st = upload(&q->d_qjl32t, st32.data(), st32.size());
+  }
+  if (st == TQ_OK) {
     // Rotation as fp16 pieces for the tensor-core encode.  Hadamard: d^1.5 R
     // is an integer matrix (exact in fp16 when every |entry| <= 2048, else
     // split into two exact pieces).  Haar: R * 2^8 split into hi + lo fp16.
@@ -509,6 +517,7 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
   kt.rot = q->d_rot;
   kt.qjl16 = q->d_qjl16;
   kt.qjl32 = q->d_qjl32;
+  kt.qjl32t = q->d_qjl32t;
   *out = q;
   return TQ_OK;
 }

@@ -22,6 +22,7 @@ struct KernelTables {
   const float *rot;                   // Haar: d x d row-major fp32 (u = R x)
   const uint16_t *qjl16;              // m x d fp16 bit patterns of S
   const float *qjl32;                 // m x d fp32 values of S (same numbers)
+  const float *qjl32t;                // d x m: S transposed (coalesced S y~ over rows)
 };
 
 }  // namespace tq
@@ -40,6 +41,7 @@ struct tq_quantizer {
   float *d_rot = nullptr;
   uint16_t *d_qjl16 = nullptr;
   float *d_qjl32 = nullptr;
+  float *d_qjl32t = nullptr;
   // tensor-core encode: R = tc_rho * (sum of tc_rot_pieces fp16 matrices)
   uint16_t *d_rot16 = nullptr;   // [pieces][d][d] fp16 bits
   int tc_rot_pieces = 0;

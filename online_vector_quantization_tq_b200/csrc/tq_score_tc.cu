@@ -406,7 +406,7 @@ k_score_tc(const ScoreTCParams p) {
     }
   }
   if (!failed && t1 > t0) {
-    const bool ok = sm100::mbar_wait(mma_bar, ph_mma, p.err, 23);
+    const bool ok = __syncthreads_and(sm100::mbar_wait(mma_bar, ph_mma, p.err, 23)) != 0;  // CTA-uniform
     sm100::tc_fence_after();
     if (ok) score_epilogue(p, sQ, tmem + lane, prev_g, prev_kin, prev_valid, prev_nr);
   }

@@ -253,16 +253,15 @@ k_prep_fwht_block(KernelTables kt, RowSource src, int64_t nq, float *ytil, float
   v[j] = x;
   ytil[row * D + j] = x;
   __syncthreads();
-  const int lane = j % 32, warp = j / 32;
-  for (int i = warp; i < D; i += D / 32) {
-    const float *srow = kt.qjl32 + (size_t)i * D;
-    float acc = 0.f;
-#pragma unroll
-    for (int k = lane; k < D; k += 32) acc = fmaf(srow[k], v[k], acc);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) p[row * D + i] = acc;
+  // p_j = sum_k S[j][k] y~_k: thread j walks column j of S^T, so every load
+  // of the warp is one contiguous segment
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < D; k += 2) {
+    acc0 = fmaf(kt.qjl32t[(size_t)k * D + j], v[k], acc0);
+    acc1 = fmaf(kt.qjl32t[(size_t)(k + 1) * D + j], v[k + 1], acc1);
   }
+  p[row * D + j] = acc0 + acc1;
 }
 
 // ============================================================ score
