@@ -14,6 +14,9 @@
 // registers, four codes per instruction); the query operand has five rows
 // per query: [yh | 0 | 0], [yl | yh | 0], [0 | yl | 0], [0 | 0 | ph],
 // [0 | 0 | pl].
+// The key operand is written straight into tensor memory (tcgen05.st) and the
+// MMA reads it from there; the query operand is stored in global memory as the
+// image of its swizzled shared-memory tile and arrives by one bulk copy.
 // Accumulation is exact in int32; the epilogue forms
 //   s = ||x|| (y.c * 2^-(sy+sc) + gamma sqrt(pi/2)/m (2 p.bits - sum p) 2^-sp)
 // (TurboQuant blog 三-四: asymmetric estimator on packed keys; TurboQuant
@@ -53,6 +56,9 @@ __host__ __device__ constexpr int sign_byte_pos(int i) { return 4 * (i % 8) + i 
 __global__ void __launch_bounds__(128)
 k_query_operand(const float *ytil, const float *p, int d, int m, int w, int64_t G, int N, int cexp,
                 float qjl_scale, int8_t *qop, float4 *qsc) {
+  // byte k of operand row n sits where the 128-byte-swizzled K-major tile
+  // (three 128-byte K atoms of N rows) keeps it in shared memory
+  auto at = [N](int n, int k) { return (k / 128) * (N * 128) + sm100::sw128_offset(n, (k % 128) / 16) + k % 16; };
   const int64_t qrow = blockIdx.x;
   const int64_t g = qrow / G, ql = qrow % G;
   const float *yr = ytil + qrow * d;
@@ -79,16 +85,16 @@ k_query_operand(const float *ytil, const float *p, int d, int m, int w, int64_t 
   frexpf(ap, &ep);
   const int sy = ay > 0.f ? 14 - ey : 0;  // |y| 2^sy < 2^14
   const int sp = ap > 0.f ? 14 - ep : 0;
-  int8_t *r0 = qop + ((g * N) + kColsPerQuery * ql) * kScoreKBytes;
-  int8_t *r1 = r0 + kScoreKBytes, *rl = r1 + kScoreKBytes, *r2 = rl + kScoreKBytes, *r3 = r2 + kScoreKBytes;
+  int8_t *img = qop + g * (int64_t)N * kScoreKBytes;
+  const int n0 = kColsPerQuery * (int)ql;  // rows n0..n0+4: yh, yl|yh, yl, ph, pl
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     const int v = __float2int_rn(ldexpf(yr[j], sy));
     const int hi = (v + 128) >> 8, lo = v - 256 * hi;
     const int k = (j / 32) * 32 + code_byte_pos(w, j % 32);
-    r0[k] = (int8_t)hi;
-    r1[k] = (int8_t)lo;
-    r1[128 + k] = (int8_t)hi;
-    rl[128 + k] = (int8_t)lo;
+    img[at(n0, k)] = (int8_t)hi;
+    img[at(n0 + 1, k)] = (int8_t)lo;
+    img[at(n0 + 1, 128 + k)] = (int8_t)hi;
+    img[at(n0 + 2, 128 + k)] = (int8_t)lo;
   }
   int psum = 0;
   for (int i = threadIdx.x; i < m; i += blockDim.x) {
@@ -96,8 +102,8 @@ k_query_operand(const float *ytil, const float *p, int d, int m, int w, int64_t 
     psum += v;
     const int hi = (v + 128) >> 8, lo = v - 256 * hi;
     const int k = 256 + (i / 32) * 32 + sign_byte_pos(i % 32);
-    r2[k] = (int8_t)hi;
-    r3[k] = (int8_t)lo;
+    img[at(n0 + 3, k)] = (int8_t)hi;
+    img[at(n0 + 4, k)] = (int8_t)lo;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
@@ -168,258 +174,295 @@ __device__ __forceinline__ void expand_codes(const uint32_t *cw, const uint32_t 
   }
 }
 
-__device__ __forceinline__ void sts128_sw(uint8_t *atom, int row, int chunk, uint32_t a, uint32_t b, uint32_t c,
-                                          uint32_t d) {
-  *reinterpret_cast<uint4 *>(atom + sm100::sw128_offset(row, chunk)) = make_uint4(a, b, c, d);
-}
 
-
-// Scores of one key (this thread's TMEM lane) for every query of its group.
-__device__ __forceinline__ void score_epilogue(const ScoreTCParams &p, const float4 *sQ, uint32_t taddr,
-                                               int64_t g, int64_t kin, bool valid, float2 nr) {
-  for (int q0 = 0; q0 < p.G; q0 += 3) {  // 15 of the 16 loaded columns = 3 queries
-    uint32_t dv[16];
-    sm100::tmem_ld16(taddr + kColsPerQuery * q0, dv);
-    sm100::tmem_wait_ld();
-#pragma unroll
-    for (int qq = 0; qq < 3; ++qq) {
-      const int q = q0 + qq;
-      if (q < p.G && valid) {
-        const float4 sc = sQ[q];
-        const int *v = reinterpret_cast<const int *>(dv) + kColsPerQuery * qq;
-        const int sb = 2 * (256 * v[3] + v[4]) - (int)sc.z;
-        const float a = fmaf((float)v[0], 65536.f, fmaf((float)v[1], 256.f, (float)v[2])) * sc.x;
-        float s = nr.x * fmaf(nr.y * sc.y, (float)sb, a);
-        float *o = p.out + (g * p.G + q) * p.ldo + kin;
-        if (p.accumulate) s += *o;
-        *o = s;
-      }
-    }
-  }
-}
 
 }  // namespace
 
 // ------------------------------------------------------------------ scorer
-// 128 threads = 128 keys per tile.  Persistent CTAs walk a contiguous range of
-// tiles (a group's tiles are contiguous).  Raw key rows (codes, sign words,
-// norms) arrive by bulk asynchronous copies into a ring of kStages shared
-// buffers, issued kStages tiles ahead; each tile is then expanded into the
-// MMA operand, multiplied, and its scores are written one tile later while
-// the next tile is being prepared.
+// Warp-specialised, one persistent CTA per SM walking a contiguous range of
+// 128-key tiles (a group's tiles are contiguous):
+//   warps 0-7   expanders, two groups of four taking alternate tiles; thread
+//               (warp % 4, lane) expands key row 32 (warp % 4) + lane into
+//               its group's key operand in TMEM;
+//   warps 8-15  epilogue, two per TMEM lane quarter, queries split between
+//               them; scores of a tile from its TMEM accumulator;
+//   warp 16     MMA issue (one thread), query operand copies, TMEM owner;
+//   warp 17     raw key rows: bulk copies into a ring of kStages buffers.
+// Hand-offs are mbarriers only: stage full/empty, key operand full/empty,
+// accumulator full/empty.  Every wait is bounded and gives up as soon as
+// another role has failed, after which all roles leave their loops, in-flight
+// copies and MMAs are waited for (bounded) and TMEM is freed.
 constexpr int kStages = 4;
+constexpr int kExpWarps = 8, kEpiWarps = 8;
+constexpr int kMmaWarp = kExpWarps + kEpiWarps, kLoadWarp = kMmaWarp + 1;
+constexpr int kScoreThreads = (kLoadWarp + 1) * 32;
+constexpr int kACols = kScoreKBytes / 4;  // TMEM columns of one key operand
+
+// TMEM plan of one CTA: accumulators (N columns + 16 for the epilogue's wide
+// loads, rounded to 32) then two key operands.
+struct ScoreTmem {
+  int npad, nacc, ncols;
+  __host__ __device__ explicit ScoreTmem(int N) {
+    npad = (N + 16 + 31) / 32 * 32;
+    nacc = 2 * npad + 2 * kACols <= 512 ? 2 : 1;
+    const int used = nacc * npad + 2 * kACols;
+    ncols = 32;
+    while (ncols < used) ncols <<= 1;
+  }
+  __host__ __device__ int acc(int b) const { return b * npad; }
+  __host__ __device__ int a(int e) const { return nacc * npad + e * kACols; }
+};
 
 template <int W, int NG>
 struct ScoreSmem {
   static constexpr int kCW = W * NG;                // code words per key
   static constexpr int kCodeBytes = 128 * kCW * 4;  // per stage
   static constexpr int kSignBytes = 128 * NG * 4;
-  static constexpr int kNormBytes = 128 * 8;
-  static constexpr int kStageBytes = kCodeBytes + kSignBytes + kNormBytes;
-  static constexpr int kOffA = 0;                          // 3 x 16 KB operand atoms
-  static constexpr int kOffStage = 3 * 16384;
-  static constexpr int kOffB = kOffStage + kStages * kStageBytes;
+  static constexpr int kStageBytes = kCodeBytes + kSignBytes;
+  static constexpr int kOffB = kStages * kStageBytes;  // multiple of 1024
+  enum Bar { kFull = 0, kEmpty = kStages, kAFull = 2 * kStages, kAEmpty = kAFull + 2, kAccFull = kAEmpty + 2,
+             kAccEmpty = kAccFull + 2, kBFull = kAccEmpty + 2, kMmaDone = kBFull + 1, kNumBars = kMmaDone + 1 };
 };
 
 template <int W, int NG, bool BULK>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kScoreThreads, 1)
 k_score_tc(const ScoreTCParams p) {
   using SM = ScoreSmem<W, NG>;
   constexpr int CW = SM::kCW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sA = smem + SM::kOffA;
-  uint8_t *sStage = smem + SM::kOffStage;
-  uint8_t *sB = smem + (BULK ? SM::kOffB : SM::kOffStage);
-  float4 *sQ = reinterpret_cast<float4 *>(sB + 3 * p.N * 128);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sQ + p.G);  // [kStages] stages, then the MMA barrier
-  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + kStages + 1);
+  uint8_t *sStage = smem;
+  uint8_t *sB = smem + (BULK ? SM::kOffB : 0);
+  const uint32_t b_bytes = (uint32_t)p.N * kScoreKBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + b_bytes);
+  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + SM::kNumBars);
+  volatile int *sAbort = reinterpret_cast<volatile int *>(sTmem + 1);
 
-  const int tid = threadIdx.x;
-  const uint32_t lane = (uint32_t)(tid & ~31) << 16;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const ScoreTmem tp(p.N);
   const int64_t t0 = (p.ntiles * blockIdx.x) / gridDim.x;
   const int64_t t1 = (p.ntiles * (blockIdx.x + 1)) / gridDim.x;
-  uint32_t ncols = 32;
-  while ((int)ncols < p.N + 16) ncols <<= 1;  // epilogue loads read 16 columns from 5*q0
+  const int n_it = (int)(t1 - t0);
+  const int64_t tpg = p.tiles_per_group;
   if (tid == 0) {
-    for (int i = 0; i <= kStages; ++i) sm100::mbar_init(&bars[i], 1);
+    for (int i = 0; i < kStages; ++i) {
+      sm100::mbar_init(&bars[SM::kFull + i], 1);
+      sm100::mbar_init(&bars[SM::kEmpty + i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&bars[SM::kAFull + i], 4);
+      sm100::mbar_init(&bars[SM::kAEmpty + i], 1);
+      sm100::mbar_init(&bars[SM::kAccFull + i], 1);
+      sm100::mbar_init(&bars[SM::kAccEmpty + i], kEpiWarps);
+    }
+    sm100::mbar_init(&bars[SM::kBFull], 1);
+    sm100::mbar_init(&bars[SM::kMmaDone], 1);
+    *sAbort = 0;
     sm100::fence_barrier_init();
   }
-  if (tid < 32) {
-    sm100::tmem_alloc(sTmem, ncols);
+  if (warp == kMmaWarp) {
+    sm100::tmem_alloc(sTmem, (uint32_t)tp.ncols);
     sm100::tmem_relinquish();
   }
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *sTmem;
-  uint64_t *mma_bar = &bars[kStages];
-  uint32_t tch[4], tcl[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    tch[k] = p.tch[k];
-    tcl[k] = p.tcl[k];
-  }
-  const uint32_t idesc = sm100::idesc_s8_s32(128, p.N);
-  const int64_t tpg = p.tiles_per_group;
-
-  // Tile t covers keys [kin0, kin0 + 128) (relative to key_base) of group
-  // t / tpg; with BULK, stage slot (t - t0) % kStages holds exactly its rows.
-  auto issue_stage = [&](int64_t t, int slot) {
-    const int64_t g = t / tpg;
-    const int64_t kin0 = (t % tpg) * 128;
-    const int64_t key0 = g * p.kpg + p.key_base + kin0;
-    const int64_t left = p.nkeys - kin0;
-    const int rows = left < 128 ? (int)left : 128;
-    uint8_t *st = sStage + slot * SM::kStageBytes;
-    const uint32_t cb = rows * CW * 4, sb = rows * NG * 4, nb = rows * 8;
-    sm100::mbar_expect_tx(&bars[slot], cb + sb + nb);
-    sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[slot]);
-    sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[slot]);
-    sm100::bulk_load(st + SM::kCodeBytes + SM::kSignBytes, p.norms + key0, nb, &bars[slot]);
+  auto wait = [&](int bar, uint32_t parity, int code) {
+    return sm100::mbar_wait_abort(&bars[bar], parity, sAbort, p.err, code);
   };
-  int64_t issued = t0;  // next tile whose stage is to be issued (thread 0)
-  if constexpr (BULK) {
-    if (tid == 0)
-      for (; issued < t1 && issued < t0 + kStages; ++issued) issue_stage(issued, (int)(issued - t0));
-  }
+  // state the teardown needs
+  int64_t issued = 0;      // stages issued (load warp)
+  int mma_issued = 0;      // tiles whose MMAs were issued (MMA thread)
+  bool b_pending = false;  // a query-operand copy not yet seen complete
+  uint32_t b_ph = 0, md_ph = 0;
 
-  uint32_t ph_mma = 0u;
-  bool failed = false;
-  int64_t cur_group = -1;
-  int64_t g = t0 / tpg, tin = t0 % tpg;  // group and tile-in-group of tile t
-  int64_t prev_g = -1, prev_kin = 0;
-  bool prev_valid = false;
-  float2 prev_nr = make_float2(0.f, 0.f);
-  int64_t t = t0;
-  for (; t < t1; ++t) {
-    const int slot = (int)((t - t0) % kStages);
-    const int64_t kin = tin * 128 + tid;
-    const bool valid = kin < p.nkeys;
-    bool ok = true;
-    // ---- raw row of this tile's key
-    uint32_t cw[CW], sw[NG];
-    float2 nr = make_float2(0.f, 0.f);
+  if (warp < kExpWarps) {
+    // ------------------------------------------------------------ expanders
+    const int e = warp / 4, quarter = warp % 4, row = 32 * quarter + lane;
+    const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
+    uint32_t tch[4], tcl[4];
 #pragma unroll
-    for (int k = 0; k < CW; ++k) cw[k] = 0u;
+    for (int k = 0; k < 4; ++k) {
+      tch[k] = p.tch[k];
+      tcl[k] = p.tcl[k];
+    }
+    for (int it = e; it < n_it; it += 2) {
+      const int64_t t = t0 + it, g = t / tpg, kin = (t % tpg) * 128 + row;
+      const bool valid = kin < p.nkeys;
+      uint32_t cw[CW], sw[NG];
 #pragma unroll
-    for (int k = 0; k < NG; ++k) sw[k] = 0u;
-    if constexpr (BULK) {
-      ok = sm100::mbar_wait(&bars[slot], (uint32_t)(((t - t0) / kStages) & 1), p.err, 21);
-      const uint8_t *st = sStage + slot * SM::kStageBytes;
-      if (valid) {
-        if constexpr (CW % 4 == 0) {
+      for (int k = 0; k < CW; ++k) cw[k] = 0u;
+#pragma unroll
+      for (int k = 0; k < NG; ++k) sw[k] = 0u;
+      if constexpr (BULK) {
+        const int slot = it % kStages;
+        if (!__all_sync(0xffffffffu, wait(SM::kFull + slot, (uint32_t)((it / kStages) & 1), 21))) break;
+        const uint8_t *st = sStage + slot * SM::kStageBytes;
+        if (valid) {
+          const uint4 *crow = reinterpret_cast<const uint4 *>(st + row * CW * 4);
 #pragma unroll
           for (int k = 0; k < CW / 4; ++k) {
-            const uint4 v = reinterpret_cast<const uint4 *>(st + tid * CW * 4)[k];
-            cw[4 * k] = v.x; cw[4 * k + 1] = v.y; cw[4 * k + 2] = v.z; cw[4 * k + 3] = v.w;
+            const uint4 v = crow[k];
+            cw[4 * k] = v.x;
+            cw[4 * k + 1] = v.y;
+            cw[4 * k + 2] = v.z;
+            cw[4 * k + 3] = v.w;
           }
-        } else {
-#pragma unroll
-          for (int k = 0; k < CW; ++k) cw[k] = reinterpret_cast<const uint32_t *>(st + tid * CW * 4)[k];
+          const uint4 sv = *reinterpret_cast<const uint4 *>(st + SM::kCodeBytes + row * NG * 4);
+          sw[0] = sv.x;
+          sw[1] = sv.y;
+          sw[2] = sv.z;
+          sw[3] = sv.w;
         }
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&bars[SM::kEmpty + slot]);
+      } else {
+        if (valid) {
+          const int64_t key = g * p.kpg + p.key_base + kin;
 #pragma unroll
-        for (int k = 0; k < NG; ++k)
-          sw[k] = reinterpret_cast<const uint32_t *>(st + SM::kCodeBytes + tid * NG * 4)[k];
-        nr = reinterpret_cast<const float2 *>(st + SM::kCodeBytes + SM::kSignBytes)[tid];
+          for (int k = 0; k < CW; ++k) cw[k] = __ldg(p.codes + key * CW + k);
+#pragma unroll
+          for (int k = 0; k < NG; ++k) sw[k] = __ldg(p.signs + key * NG + k);
+        }
       }
-    } else {
-      if (valid) {
-        const int64_t key = g * p.kpg + p.key_base + kin;
-#pragma unroll
-        for (int k = 0; k < CW; ++k) cw[k] = __ldg(p.codes + key * CW + k);
-#pragma unroll
-        for (int k = 0; k < NG; ++k) sw[k] = __ldg(p.signs + key * NG + k);
-        nr = __ldg(p.norms + key);
-      }
-    }
-    // ---- expand into registers
-    uint32_t ach[NG][8], acl[NG][8], abt[NG][8];
-#pragma unroll
-    for (int gi = 0; gi < NG; ++gi) {
-      expand_codes<W>(cw + gi * W, tch, tcl, ach[gi], acl[gi]);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) abt[gi][k] = (sw[gi] >> k) & 0x01010101u;
-    }
-    // ---- scores of the previous tile
-    if (t > t0) {
-      ok = sm100::mbar_wait(mma_bar, ph_mma, p.err, 22) && ok;
-      ph_mma ^= 1u;
+      // the key operand buffer was last read by the MMAs of tile it - 2
+      const int use = it / 2;
+      if (use > 0 && !__all_sync(0xffffffffu, wait(SM::kAEmpty + e, (uint32_t)((use - 1) & 1), 22))) break;
       sm100::tc_fence_after();
-      score_epilogue(p, sQ, tmem + lane, prev_g, prev_kin, prev_valid, prev_nr);
-    }
-    // ---- the query operand of this group
-    if (g != cur_group) {
+      const uint32_t ta = tmem + tlane + (uint32_t)tp.a(e);
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+        uint32_t ch[8], cl[8], bt[8];
+        expand_codes<W>(cw + gi * W, tch, tcl, ch, cl);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) bt[k] = (sw[gi] >> k) & 0x01010101u;
+        sm100::tmem_st8(ta + 8 * gi, ch);
+        sm100::tmem_st8(ta + 32 + 8 * gi, cl);
+        sm100::tmem_st8(ta + 64 + 8 * gi, bt);
+      }
+      sm100::tmem_wait_st();
       sm100::tc_fence_before();
-      __syncthreads();
-      const int8_t *src = p.qop + g * (int64_t)p.N * kScoreKBytes;
-      for (int i = tid; i < p.N * 24; i += 128) {  // 16-byte chunks
-        const int n = i / 24, c = i % 24;
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src + n * kScoreKBytes) + c);
-        *reinterpret_cast<uint4 *>(sB + (c / 8) * (p.N * 128) + sm100::sw128_offset(n, c % 8)) = v;
-      }
-      for (int i = tid; i < p.G; i += 128) sQ[i] = p.qsc[g * p.G + i];
-      cur_group = g;
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&bars[SM::kAFull + e]);
     }
-    // ---- key operand row
+  } else if (warp < kMmaWarp) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp % 4, eh = (warp - kExpWarps) / 4, row = 32 * quarter + lane;
+    const int q_half = (int)((p.G + 1) / 2);
+    const int q_lo = eh ? q_half : 0, q_hi = eh ? (int)p.G : q_half;
+    const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
+    for (int it = 0; it < n_it; ++it) {
+      const int64_t t = t0 + it, g = t / tpg, kin = (t % tpg) * 128 + row;
+      const bool valid = kin < p.nkeys;
+      float2 nr = make_float2(0.f, 0.f);
+      if (valid) nr = __ldg(p.norms + g * p.kpg + p.key_base + kin);
+      const int ab = it % tp.nacc, use = it / tp.nacc;
+      if (!__all_sync(0xffffffffu, wait(SM::kAccFull + ab, (uint32_t)(use & 1), 23))) break;
+      sm100::tc_fence_after();
+      const uint32_t taddr = tmem + tlane + (uint32_t)tp.acc(ab);
+      const float4 *qs = p.qsc + g * p.G;
+      float *orow = p.out + g * p.G * p.ldo + kin;
+      for (int q0 = q_lo; q0 < q_hi; q0 += 3) {  // 15 of 16 loaded columns = 3 queries
+        uint32_t dv[16];
+        sm100::tmem_ld16(taddr + kColsPerQuery * q0, dv);
+        float4 sc[3];
 #pragma unroll
-    for (int gi = 0; gi < NG; ++gi) {
-      sts128_sw(sA, tid, 2 * gi, ach[gi][0], ach[gi][1], ach[gi][2], ach[gi][3]);
-      sts128_sw(sA, tid, 2 * gi + 1, ach[gi][4], ach[gi][5], ach[gi][6], ach[gi][7]);
-      sts128_sw(sA + 16384, tid, 2 * gi, acl[gi][0], acl[gi][1], acl[gi][2], acl[gi][3]);
-      sts128_sw(sA + 16384, tid, 2 * gi + 1, acl[gi][4], acl[gi][5], acl[gi][6], acl[gi][7]);
-      sts128_sw(sA + 32768, tid, 2 * gi, abt[gi][0], abt[gi][1], abt[gi][2], abt[gi][3]);
-      sts128_sw(sA + 32768, tid, 2 * gi + 1, abt[gi][4], abt[gi][5], abt[gi][6], abt[gi][7]);
-    }
-    sm100::fence_proxy_async();
-    sm100::tc_fence_before();
-    failed |= __syncthreads_or(!ok || failed) != 0;
-    if (failed) break;
-    sm100::tc_fence_after();
-    if (tid == 0) {
-      const uint32_t a0 = sm100::smem_u32(sA), b0 = sm100::smem_u32(sB);
-      // coordinates beyond d (NG < 4) meet zero query bytes, so the unwritten
-      // part of the key row does not contribute
+        for (int qq = 0; qq < 3; ++qq) sc[qq] = q0 + qq < q_hi ? __ldg(qs + q0 + qq) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sm100::tmem_wait_ld();
 #pragma unroll
-      for (int ks = 0; ks < kScoreKBytes / 32; ++ks) {
-        const int atom = ks / 4, off = (ks % 4) * 32;
-        const uint64_t a = sm100::desc_sw128(a0 + atom * 16384 + off);
-        const uint64_t b = sm100::desc_sw128(b0 + atom * (p.N * 128) + off);
-        sm100::mma_i8(tmem, a, b, idesc, ks != 0);
-      }
-      sm100::mma_commit(mma_bar);
-      // every thread has read this tile's stage: refill it kStages tiles ahead
-      if constexpr (BULK) {
-        if (issued < t1) {
-          issue_stage(issued, slot);
-          ++issued;
+        for (int qq = 0; qq < 3; ++qq) {
+          const int q = q0 + qq;
+          if (q < q_hi && valid) {
+            const int *v = reinterpret_cast<const int *>(dv) + kColsPerQuery * qq;
+            const int sb = 2 * (256 * v[3] + v[4]) - (int)sc[qq].z;
+            const float a = fmaf((float)v[0], 65536.f, fmaf((float)v[1], 256.f, (float)v[2])) * sc[qq].x;
+            float sres = nr.x * fmaf(nr.y * sc[qq].y, (float)sb, a);
+            float *o = orow + q * p.ldo;
+            if (p.accumulate) sres += *o;
+            *o = sres;
+          }
         }
       }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&bars[SM::kAccEmpty + ab]);
     }
-    prev_g = g;
-    prev_kin = kin;
-    prev_valid = valid;
-    prev_nr = nr;
-    if (++tin == tpg) {
-      tin = 0;
-      ++g;
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = sm100::idesc_s8_s32(128, p.N);
+      const uint32_t b0 = sm100::smem_u32(sB);
+      int64_t cur_group = -1;
+      for (int it = 0; it < n_it; ++it) {
+        const int64_t g = (t0 + it) / tpg;
+        if (g != cur_group) {
+          if (it > 0) {  // every MMA reading the old query operand has completed
+            sm100::mma_commit(&bars[SM::kMmaDone]);
+            const bool ok = wait(SM::kMmaDone, md_ph, 24);
+            md_ph ^= 1u;
+            if (!ok) break;
+          }
+          sm100::mbar_expect_tx(&bars[SM::kBFull], b_bytes);
+          sm100::bulk_load(sB, p.qop + g * (int64_t)b_bytes, b_bytes, &bars[SM::kBFull]);
+          b_pending = true;
+          if (!wait(SM::kBFull, b_ph, 25)) break;
+          b_ph ^= 1u;
+          b_pending = false;
+          cur_group = g;
+        }
+        const int e = it & 1, ab = it % tp.nacc;
+        if (!wait(SM::kAFull + e, (uint32_t)((it / 2) & 1), 26)) break;
+        if (it >= tp.nacc && !wait(SM::kAccEmpty + ab, (uint32_t)((it / tp.nacc - 1) & 1), 27)) break;
+        sm100::tc_fence_after();
+        const uint32_t ta = tmem + (uint32_t)tp.a(e), td = tmem + (uint32_t)tp.acc(ab);
+        bool first = true;
+#pragma unroll
+        for (int ks = 0; ks < kScoreKBytes / 32; ++ks) {
+          if (ks % 4 >= NG) continue;  // coordinates beyond d
+          const uint64_t db = sm100::desc_sw128(b0 + (ks / 4) * (p.N * 128) + (ks % 4) * 32);
+          sm100::mma_i8_ts(td, ta + 8 * ks, db, idesc, !first);
+          first = false;
+        }
+        sm100::mma_commit(&bars[SM::kAEmpty + e]);
+        sm100::mma_commit(&bars[SM::kAccFull + ab]);
+        mma_issued = it + 1;
+      }
+    }
+  } else if (BULK && lane == 0) {
+    // ------------------------------------------------------------ raw key rows
+    for (; issued < n_it; ++issued) {
+      const int j = (int)issued, slot = j % kStages;
+      if (j >= kStages && !wait(SM::kEmpty + slot, (uint32_t)((j / kStages - 1) & 1), 28)) break;
+      const int64_t t = t0 + j, g = t / tpg, kin0 = (t % tpg) * 128;
+      const int64_t key0 = g * p.kpg + p.key_base + kin0;
+      const int64_t left = p.nkeys - kin0;
+      const int rows = left < 128 ? (int)left : 128;
+      uint8_t *st = sStage + slot * SM::kStageBytes;
+      const uint32_t cb = rows * CW * 4, sb = rows * NG * 4;
+      sm100::mbar_expect_tx(&bars[SM::kFull + slot], cb + sb);
+      sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
+      sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
     }
   }
-  if (!failed && t1 > t0) {
-    const bool ok = __syncthreads_and(sm100::mbar_wait(mma_bar, ph_mma, p.err, 23)) != 0;  // CTA-uniform
-    sm100::tc_fence_after();
-    if (ok) score_epilogue(p, sQ, tmem + lane, prev_g, prev_kin, prev_valid, prev_nr);
-  }
-  if constexpr (BULK) {
-    if (failed && tid == 0) {
-      // bounded wait for stage copies issued but not consumed
-      for (int64_t u = t + 1; u < issued; ++u)
-        sm100::mbar_wait(&bars[(u - t0) % kStages], (uint32_t)(((u - t0) / kStages) & 1), p.err, 24);
+  // ------------------------------------------------------------ teardown
+  __syncthreads();
+  if (warp == kMmaWarp && lane == 0) {
+    if (mma_issued > 0) {  // no MMA may still write TMEM when it is freed
+      sm100::mma_commit(&bars[SM::kMmaDone]);
+      sm100::mbar_wait(&bars[SM::kMmaDone], md_ph, p.err, 29);
     }
+    if (b_pending) sm100::mbar_wait(&bars[SM::kBFull], b_ph, p.err, 30);
+  }
+  if (BULK && warp == kLoadWarp && lane == 0 && *sAbort) {
+    // copies issued but possibly not consumed: the last kStages issued
+    for (int64_t j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+      sm100::mbar_wait(&bars[SM::kFull + j % kStages], (uint32_t)((j / kStages) & 1), p.err, 31);
   }
   sm100::tc_fence_before();
   __syncthreads();
-  if (tid < 32) sm100::tmem_dealloc(tmem, ncols);
+  sm100::tc_fence_after();
+  if (warp == kMmaWarp) sm100::tmem_dealloc(tmem, (uint32_t)tp.ncols);
 }
 
 // ------------------------------------------------------------------ host side
@@ -471,25 +514,24 @@ tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, in
   prm.accumulate = accumulate;
   prm.err = q->d_err;
   const int ng = q->d / 32, cwords = q->w * ng;
-  const size_t stage_bytes = (size_t)128 * (cwords + ng) * 4 + 128 * 8;
-  // bulk copies need 16-byte multiples and 16-byte aligned rows for every tile
-  const bool bulk = ng == 4 && kpg % 2 == 0 && key_base % 2 == 0 && nkeys % 2 == 0 &&
-                    reinterpret_cast<uintptr_t>(norms) % 16 == 0 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
+  const size_t stage_bytes = (size_t)128 * (cwords + ng) * 4;
+  // bulk copies need 16-byte aligned starts and sizes: with d = 128 a key's
+  // code and sign rows are multiples of 16 bytes, so any tile qualifies
+  const bool bulk = ng == 4 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
                     reinterpret_cast<uintptr_t>(signs) % 16 == 0;
-  const size_t smem = 1024 + 3 * 16384 + (bulk ? kStages * stage_bytes : 0) + 3 * (size_t)N * 128 +
-                      (size_t)G * 16 + 128;
+  if (reinterpret_cast<uintptr_t>(qop) % 16 != 0) return TQ_ERR_ALIGNMENT;
+  const size_t smem = 1024 + (bulk ? kStages * stage_bytes : 0) + (size_t)N * kScoreKBytes + 8 * 24 + 16;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (228 * 1024) / (smem + 1024)));
-  const int64_t grid = std::min<int64_t>(prm.ntiles, (int64_t)sms * per_sm);
+  const int64_t grid = std::min<int64_t>(prm.ntiles, (int64_t)sms);
   if (grid <= 0) return TQ_OK;
 #define TQ_SC(WW, NGG)                                                                                   \
   {                                                                                                      \
     auto kern = bulk ? k_score_tc<WW, NGG, (NGG == 4)> : k_score_tc<WW, NGG, false>;                     \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
       return TQ_ERR_CUDA;                                                                                \
-    kern<<<(unsigned)grid, 128, smem, st>>>(prm);                                                        \
+    kern<<<(unsigned)grid, kScoreThreads, smem, st>>>(prm);                                                        \
     break;                                                                                               \
   }
 #define TQ_SC_NG(WW)                     \

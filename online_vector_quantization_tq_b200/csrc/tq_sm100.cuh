@@ -1,9 +1,9 @@
 // Thin inline-PTX wrappers for the sm_100a features the tensor-core kernels
 // use: mbarriers, TMA tiled loads, tcgen05 (TMEM allocation, MMA, commit,
 // TMEM loads) and the shared-memory operand descriptors.  Every wait on an
-// mbarrier is bounded: after kSpinLimit polls it records an error code in
-// a device word and reports failure, so a broken pipeline ends the kernel
-// instead of hanging the GPU.
+// mbarrier is bounded (about 2 s of suspended polling): on timeout it records
+// an error code in a device word and reports failure, so a broken pipeline
+// ends the kernel instead of hanging the GPU.
 #pragma once
 
 #include <cuda.h>
@@ -14,7 +14,6 @@
 namespace tq {
 namespace sm100 {
 
-constexpr uint32_t kSpinLimit = 1u << 26;  // ~seconds of polling
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -42,13 +41,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `ns` nanoseconds pass, instead of spinning on the issue
+// slots other warps need.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t *bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+constexpr uint32_t kWaitSliceNs = 1000000;  // one sleep of at most 1 ms
+constexpr uint32_t kWaitSlices = 2000;      // about 2 s in all
+
 // Bounded wait; on timeout writes `code` to *err (if not yet set) and
 // returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  for (uint32_t i = 0; i < kWaitSlices; ++i)
+    if (mbar_try_wait_for(bar, parity, kWaitSliceNs)) return true;
   atomicCAS(err, 0, code);
   return false;
+}
+
+// Bounded wait that also gives up as soon as another role of the CTA has
+// raised *abort; on its own timeout it records `code` and raises *abort.
+__device__ __forceinline__ bool mbar_wait_abort(uint64_t *bar, uint32_t parity, volatile int *abort, int *err,
+                                                int code) {
+  for (uint32_t i = 0; i < kWaitSlices; ++i) {
+    if (mbar_try_wait_for(bar, parity, kWaitSliceNs)) return true;
+    if (*abort) return false;
+  }
+  atomicCAS(err, 0, code);
+  *abort = 1;
+  return false;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void fence_barrier_init() {
@@ -116,6 +149,18 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_
 }
 
 // Arrives once on `bar` when all previously issued MMAs of this thread complete.
+// Same, with the A operand (128 rows x 32 bytes, K-major) read from TMEM:
+// row r in lane r, four consecutive K bytes per 32-bit column.
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
@@ -151,6 +196,12 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // One 32-bit column per lane: thread i of the warp writes lane (base + i).
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+// Thread i of the warp writes lane (base lane + i), columns [col, col+8).
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
