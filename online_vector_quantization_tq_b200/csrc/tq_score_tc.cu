@@ -181,36 +181,69 @@ __device__ __forceinline__ void expand_codes(const uint32_t *cw, const uint32_t 
 // ------------------------------------------------------------------ scorer
 // Warp-specialised, one persistent CTA per SM walking a contiguous range of
 // 128-key tiles (a group's tiles are contiguous):
-//   warps 0-7   expanders, two groups of four taking alternate tiles; thread
-//               (warp % 4, lane) expands key row 32 (warp % 4) + lane into
-//               its group's key operand in TMEM;
-//   warps 8-15  epilogue, two per TMEM lane quarter, queries split between
-//               them; scores of a tile from its TMEM accumulator;
-//   warp 16     MMA issue (one thread), query operand copies, TMEM owner;
-//   warp 17     raw key rows: bulk copies into a ring of kStages buffers.
-// Hand-offs are mbarriers only: stage full/empty, key operand full/empty,
-// accumulator full/empty.  Every wait is bounded and gives up as soon as
-// another role has failed, after which all roles leave their loops, in-flight
-// copies and MMAs are waited for (bounded) and TMEM is freed.
+//   warps 0-7    expanders, two groups of four taking alternate tiles; thread
+//                (warp % 4, lane) expands key row 32 (warp % 4) + lane into
+//                its group's key operand in TMEM;
+//   warps 8-15   epilogue, two per TMEM lane quarter, queries split between
+//                them; scores of a tile from its TMEM accumulator;
+//   warps 16-17  MMA issue, one thread each, alternate tiles (a single issuer
+//                when only one accumulator fits): an issuing thread spends
+//                tens of cycles per tcgen05 instruction, so two of them keep
+//                the tensor core fed;
+//   warp 18      bulk copies: raw key rows into a ring of kStages buffers, and
+//                each group's query operand into a ring of two.
+// Hand-offs are mbarriers only.  Every wait is bounded and gives up as soon
+// as another role has failed, after which all roles leave their loops,
+// in-flight copies and MMAs are waited for (bounded) and TMEM is freed.
 constexpr int kStages = 4;
 constexpr int kExpWarps = 8, kEpiWarps = 8;
-constexpr int kMmaWarp = kExpWarps + kEpiWarps, kLoadWarp = kMmaWarp + 1;
+constexpr int kMmaWarp = kExpWarps + kEpiWarps;  // and kMmaWarp + 1: the two MMA issuers
+constexpr int kLoadWarp = kMmaWarp + 2;
 constexpr int kScoreThreads = (kLoadWarp + 1) * 32;
 constexpr int kACols = kScoreKBytes / 4;  // TMEM columns of one key operand
 
-// TMEM plan of one CTA: accumulators (N columns + 16 for the epilogue's wide
-// loads, rounded to 32) then two key operands.
+// TMEM plan of one CTA: nacc accumulators of N columns (rounded to 32), then
+// 32 columns of slack when the epilogue's 16-column loads of the last queries
+// reach past an accumulator, then nab key operands.  Where columns allow,
+// four accumulators (the MMAs of a tile need not wait for the scores of the
+// tile two before) and two key operands per expander group (a group fills
+// one while the MMAs read the other).
 struct ScoreTmem {
-  int npad, nacc, ncols;
-  __host__ __device__ explicit ScoreTmem(int N) {
-    npad = (N + 16 + 31) / 32 * 32;
-    nacc = 2 * npad + 2 * kACols <= 512 ? 2 : 1;
-    const int used = nacc * npad + 2 * kACols;
+  int stride, lgacc, nacc, nab, dcols, ncols;
+  __host__ __device__ ScoreTmem(int N, int64_t G) {
+    stride = (N + 31) / 32 * 32;
+    const int slack = kColsPerQuery * (int)G + 11 > stride ? 32 : 0;
+    auto fit = [&](int na, int nb) { return na * stride + slack + nb * kACols <= 512; };
+    if (fit(4, 4)) {
+      lgacc = 2;
+      nab = 4;
+    } else {
+      lgacc = fit(2, 2) ? 1 : 0;
+      nab = fit(1 << lgacc, 4) ? 4 : 2;
+    }
+    nacc = 1 << lgacc;
+    dcols = nacc * stride + slack;
+    const int used = dcols + nab * kACols;
     ncols = 32;
     while (ncols < used) ncols <<= 1;
   }
-  __host__ __device__ int acc(int b) const { return b * npad; }
-  __host__ __device__ int a(int e) const { return nacc * npad + e * kACols; }
+  __host__ __device__ int acc(int b) const { return b * stride; }
+  __host__ __device__ int a(int e) const { return dcols + e * kACols; }
+};
+
+// (group, tile in group) of a walk over the CTA's tiles with a fixed stride,
+// advanced without 64-bit division.
+struct TileWalk {
+  int64_t g, tin, tpg;
+  __device__ TileWalk(int64_t t, int64_t tiles_per_group) : g(t / tiles_per_group), tin(t % tiles_per_group),
+                                                            tpg(tiles_per_group) {}
+  __device__ void advance(int stride) {
+    tin += stride;
+    while (tin >= tpg) {
+      tin -= tpg;
+      ++g;
+    }
+  }
 };
 
 template <int W, int NG>
@@ -220,8 +253,9 @@ struct ScoreSmem {
   static constexpr int kSignBytes = 128 * NG * 4;
   static constexpr int kStageBytes = kCodeBytes + kSignBytes;
   static constexpr int kOffB = kStages * kStageBytes;  // multiple of 1024
-  enum Bar { kFull = 0, kEmpty = kStages, kAFull = 2 * kStages, kAEmpty = kAFull + 2, kAccFull = kAEmpty + 2,
-             kAccEmpty = kAccFull + 2, kBFull = kAccEmpty + 2, kMmaDone = kBFull + 1, kNumBars = kMmaDone + 1 };
+  enum Bar { kFull = 0, kEmpty = kStages, kAFull = 2 * kStages, kAEmpty = kAFull + 4, kAccFull = kAEmpty + 4,
+             kAccEmpty = kAccFull + 4, kBFull = kAccEmpty + 4, kBEmpty = kBFull + 2, kMmaDone = kBEmpty + 2,
+             kNumBars = kMmaDone + 2 };
 };
 
 template <int W, int NG, bool BULK>
@@ -233,30 +267,37 @@ k_score_tc(const ScoreTCParams p) {
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sStage = smem;
   uint8_t *sB = smem + (BULK ? SM::kOffB : 0);
-  const uint32_t b_bytes = (uint32_t)p.N * kScoreKBytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + b_bytes);
+  const uint32_t b_bytes = (uint32_t)p.N * kScoreKBytes;  // one query operand
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 2 * b_bytes);
   uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + SM::kNumBars);
   volatile int *sAbort = reinterpret_cast<volatile int *>(sTmem + 1);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const ScoreTmem tp(p.N);
+  const ScoreTmem tp(p.N, p.G);
   const int64_t t0 = (p.ntiles * blockIdx.x) / gridDim.x;
   const int64_t t1 = (p.ntiles * (blockIdx.x + 1)) / gridDim.x;
   const int n_it = (int)(t1 - t0);
   const int64_t tpg = p.tiles_per_group;
+  const int64_t g0 = t0 / tpg;  // groups are counted from the CTA's first one
+  const int nis = tp.nacc >= 2 ? 2 : 1;  // MMA issuers
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       sm100::mbar_init(&bars[SM::kFull + i], 1);
       sm100::mbar_init(&bars[SM::kEmpty + i], 4);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       sm100::mbar_init(&bars[SM::kAFull + i], 4);
       sm100::mbar_init(&bars[SM::kAEmpty + i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
       sm100::mbar_init(&bars[SM::kAccFull + i], 1);
       sm100::mbar_init(&bars[SM::kAccEmpty + i], kEpiWarps);
     }
-    sm100::mbar_init(&bars[SM::kBFull], 1);
-    sm100::mbar_init(&bars[SM::kMmaDone], 1);
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&bars[SM::kBFull + i], 1);
+      sm100::mbar_init(&bars[SM::kBEmpty + i], nis);
+      sm100::mbar_init(&bars[SM::kMmaDone + i], 1);
+    }
     *sAbort = 0;
     sm100::fence_barrier_init();
   }
@@ -272,10 +313,9 @@ k_score_tc(const ScoreTCParams p) {
     return sm100::mbar_wait_abort(&bars[bar], parity, sAbort, p.err, code);
   };
   // state the teardown needs
-  int64_t issued = 0;      // stages issued (load warp)
-  int mma_issued = 0;      // tiles whose MMAs were issued (MMA thread)
-  bool b_pending = false;  // a query-operand copy not yet seen complete
-  uint32_t b_ph = 0, md_ph = 0;
+  int64_t issued = 0;  // stages issued (load warp)
+  int b_loaded = 0;    // query operands issued (load warp)
+  int mma_issued = 0;  // tiles whose MMAs this thread issued (MMA issuers)
 
   if (warp < kExpWarps) {
     // ------------------------------------------------------------ expanders
@@ -287,8 +327,9 @@ k_score_tc(const ScoreTCParams p) {
       tch[k] = p.tch[k];
       tcl[k] = p.tcl[k];
     }
-    for (int it = e; it < n_it; it += 2) {
-      const int64_t t = t0 + it, g = t / tpg, kin = (t % tpg) * 128 + row;
+    TileWalk tw(t0 + e, tpg);
+    for (int it = e; it < n_it; it += 2, tw.advance(2)) {
+      const int64_t g = tw.g, kin = tw.tin * 128 + row;
       const bool valid = kin < p.nkeys;
       uint32_t cw[CW], sw[NG];
 #pragma unroll
@@ -326,11 +367,11 @@ k_score_tc(const ScoreTCParams p) {
           for (int k = 0; k < NG; ++k) sw[k] = __ldg(p.signs + key * NG + k);
         }
       }
-      // the key operand buffer was last read by the MMAs of tile it - 2
-      const int use = it / 2;
-      if (use > 0 && !__all_sync(0xffffffffu, wait(SM::kAEmpty + e, (uint32_t)((use - 1) & 1), 22))) break;
+      // key operand buffer it % nab was last read by the MMAs of tile it - nab
+      const int ea = tp.nab == 4 ? (it & 3) : (it & 1), use = tp.nab == 4 ? (it >> 2) : (it >> 1);
+      if (use > 0 && !__all_sync(0xffffffffu, wait(SM::kAEmpty + ea, (uint32_t)((use - 1) & 1), 22))) break;
       sm100::tc_fence_after();
-      const uint32_t ta = tmem + tlane + (uint32_t)tp.a(e);
+      const uint32_t ta = tmem + tlane + (uint32_t)tp.a(ea);
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi) {
         uint32_t ch[8], cl[8], bt[8];
@@ -344,7 +385,7 @@ k_score_tc(const ScoreTCParams p) {
       sm100::tmem_wait_st();
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&bars[SM::kAFull + e]);
+      if (lane == 0) sm100::mbar_arrive(&bars[SM::kAFull + ea]);
     }
   } else if (warp < kMmaWarp) {
     // ------------------------------------------------------------ epilogue
@@ -352,17 +393,60 @@ k_score_tc(const ScoreTCParams p) {
     const int q_half = (int)((p.G + 1) / 2);
     const int q_lo = eh ? q_half : 0, q_hi = eh ? (int)p.G : q_half;
     const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
-    for (int it = 0; it < n_it; ++it) {
-      const int64_t t = t0 + it, g = t / tpg, kin = (t % tpg) * 128 + row;
+    // the norms of a tile are loaded two tiles ahead: the accumulator is often
+    // ready by the time the epilogue gets to it, so the load would not hide
+    auto norms_of = [&](const TileWalk &w, int i) {
+      const int64_t k = w.tin * 128 + row;
+      return i < n_it && k < p.nkeys ? __ldg(p.norms + w.g * p.kpg + p.key_base + k) : make_float2(0.f, 0.f);
+    };
+    TileWalk tw(t0, tpg), tw2(t0, tpg);
+    float2 nr_next = norms_of(tw2, 0);
+    tw2.advance(1);
+    float2 nr_next2 = norms_of(tw2, 1);
+    tw2.advance(1);
+    for (int it = 0; it < n_it; ++it, tw.advance(1), tw2.advance(1)) {
+      const int64_t g = tw.g, kin = tw.tin * 128 + row;
       const bool valid = kin < p.nkeys;
-      float2 nr = make_float2(0.f, 0.f);
-      if (valid) nr = __ldg(p.norms + g * p.kpg + p.key_base + kin);
-      const int ab = it % tp.nacc, use = it / tp.nacc;
+      const float2 nr = nr_next;
+      nr_next = nr_next2;
+      nr_next2 = norms_of(tw2, it + 2);
+      const int ab = it & (tp.nacc - 1), use = it >> tp.lgacc;
       if (!__all_sync(0xffffffffu, wait(SM::kAccFull + ab, (uint32_t)(use & 1), 23))) break;
       sm100::tc_fence_after();
       const uint32_t taddr = tmem + tlane + (uint32_t)tp.acc(ab);
       const float4 *qs = p.qsc + g * p.G;
       float *orow = p.out + g * p.G * p.ldo + kin;
+      auto score = [&](const uint32_t *dv, const float4 &sc) {
+        const int *v = reinterpret_cast<const int *>(dv);
+        const int sb = 2 * (256 * v[3] + v[4]) - (int)sc.z;
+        const float a = fmaf((float)v[0], 65536.f, fmaf((float)v[1], 256.f, (float)v[2])) * sc.x;
+        return nr.x * fmaf(nr.y * sc.y, (float)sb, a);
+      };
+      auto put = [&](int q, float sres) {
+        float *o = orow + q * p.ldo;
+        if (p.accumulate) sres += *o;
+        *o = sres;
+      };
+      if (q_hi - q_lo <= 6) {
+        // at most six queries: take the columns, free the accumulator, then score
+        uint32_t d0[16], d1[16];
+        float4 sc[6];
+        sm100::tmem_ld16(taddr + kColsPerQuery * q_lo, d0);
+        if (q_hi - q_lo > 3) sm100::tmem_ld16(taddr + kColsPerQuery * (q_lo + 3), d1);
+#pragma unroll
+        for (int qq = 0; qq < 6; ++qq)
+          sc[qq] = q_lo + qq < q_hi ? __ldg(qs + q_lo + qq) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sm100::tmem_wait_ld();
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&bars[SM::kAccEmpty + ab]);
+        if (valid) {
+#pragma unroll
+          for (int qq = 0; qq < 6; ++qq)
+            if (q_lo + qq < q_hi) put(q_lo + qq, score(qq < 3 ? d0 + kColsPerQuery * qq : d1 + kColsPerQuery * (qq - 3), sc[qq]));
+        }
+        continue;
+      }
       for (int q0 = q_lo; q0 < q_hi; q0 += 3) {  // 15 of 16 loaded columns = 3 queries
         uint32_t dv[16];
         sm100::tmem_ld16(taddr + kColsPerQuery * q0, dv);
@@ -370,94 +454,104 @@ k_score_tc(const ScoreTCParams p) {
 #pragma unroll
         for (int qq = 0; qq < 3; ++qq) sc[qq] = q0 + qq < q_hi ? __ldg(qs + q0 + qq) : make_float4(0.f, 0.f, 0.f, 0.f);
         sm100::tmem_wait_ld();
+        if (valid) {
 #pragma unroll
-        for (int qq = 0; qq < 3; ++qq) {
-          const int q = q0 + qq;
-          if (q < q_hi && valid) {
-            const int *v = reinterpret_cast<const int *>(dv) + kColsPerQuery * qq;
-            const int sb = 2 * (256 * v[3] + v[4]) - (int)sc[qq].z;
-            const float a = fmaf((float)v[0], 65536.f, fmaf((float)v[1], 256.f, (float)v[2])) * sc[qq].x;
-            float sres = nr.x * fmaf(nr.y * sc[qq].y, (float)sb, a);
-            float *o = orow + q * p.ldo;
-            if (p.accumulate) sres += *o;
-            *o = sres;
-          }
+          for (int qq = 0; qq < 3; ++qq)
+            if (q0 + qq < q_hi) put(q0 + qq, score(dv + kColsPerQuery * qq, sc[qq]));
         }
       }
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&bars[SM::kAccEmpty + ab]);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp < kLoadWarp) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
+    const int e = warp - kMmaWarp;
+    if (lane == 0 && e < nis) {
       const uint32_t idesc = sm100::idesc_s8_s32(128, p.N);
-      const uint32_t b0 = sm100::smem_u32(sB);
-      int64_t cur_group = -1;
-      for (int it = 0; it < n_it; ++it) {
-        const int64_t g = (t0 + it) / tpg;
-        if (g != cur_group) {
-          if (it > 0) {  // every MMA reading the old query operand has completed
-            sm100::mma_commit(&bars[SM::kMmaDone]);
-            const bool ok = wait(SM::kMmaDone, md_ph, 24);
-            md_ph ^= 1u;
-            if (!ok) break;
+      uint64_t bdesc[kScoreKBytes / 32];  // K-steps of the current query operand
+      int jcur = 0;                       // group (from g0) of the operand held
+      bool have_b = false, used = false;
+      TileWalk tw(t0 + e, tpg);
+      for (int it = e; it < n_it; it += nis, tw.advance(nis)) {
+        const int j = (int)(tw.g - g0);
+        if (!have_b || j != jcur) {
+          // release the operands of groups passed (committed: freed when this
+          // thread's MMAs reading them complete), then take the new one
+          for (int jj = jcur; jj < j; ++jj) {
+            if (jj == jcur && used)
+              sm100::mma_commit(&bars[SM::kBEmpty + (jj & 1)]);
+            else
+              sm100::mbar_arrive(&bars[SM::kBEmpty + (jj & 1)]);
           }
-          sm100::mbar_expect_tx(&bars[SM::kBFull], b_bytes);
-          sm100::bulk_load(sB, p.qop + g * (int64_t)b_bytes, b_bytes, &bars[SM::kBFull]);
-          b_pending = true;
-          if (!wait(SM::kBFull, b_ph, 25)) break;
-          b_ph ^= 1u;
-          b_pending = false;
-          cur_group = g;
+          jcur = j;
+          used = false;
+          if (!wait(SM::kBFull + (j & 1), (uint32_t)((j >> 1) & 1), 24)) break;
+          have_b = true;
+          const uint32_t b0 = sm100::smem_u32(sB + (j & 1) * b_bytes);
+#pragma unroll
+          for (int ks = 0; ks < kScoreKBytes / 32; ++ks)
+            bdesc[ks] = sm100::desc_sw128(b0 + (ks / 4) * (p.N * 128) + (ks % 4) * 32);
         }
-        const int e = it & 1, ab = it % tp.nacc;
-        if (!wait(SM::kAFull + e, (uint32_t)((it / 2) & 1), 26)) break;
-        if (it >= tp.nacc && !wait(SM::kAccEmpty + ab, (uint32_t)((it / tp.nacc - 1) & 1), 27)) break;
+        const int ea = tp.nab == 4 ? (it & 3) : (it & 1), auses = tp.nab == 4 ? (it >> 2) : (it >> 1);
+        const int ab = it & (tp.nacc - 1), ause = it >> tp.lgacc;
+        if (!wait(SM::kAFull + ea, (uint32_t)(auses & 1), 26)) break;
+        if (ause > 0 && !wait(SM::kAccEmpty + ab, (uint32_t)((ause - 1) & 1), 27)) break;
         sm100::tc_fence_after();
-        const uint32_t ta = tmem + (uint32_t)tp.a(e), td = tmem + (uint32_t)tp.acc(ab);
-        bool first = true;
+        const uint32_t ta = tmem + (uint32_t)tp.a(ea), td = tmem + (uint32_t)tp.acc(ab);
 #pragma unroll
         for (int ks = 0; ks < kScoreKBytes / 32; ++ks) {
           if (ks % 4 >= NG) continue;  // coordinates beyond d
-          const uint64_t db = sm100::desc_sw128(b0 + (ks / 4) * (p.N * 128) + (ks % 4) * 32);
-          sm100::mma_i8_ts(td, ta + 8 * ks, db, idesc, !first);
-          first = false;
+          sm100::mma_i8_ts(td, ta + 8 * ks, bdesc[ks], idesc, ks != 0);
         }
-        sm100::mma_commit(&bars[SM::kAEmpty + e]);
+        sm100::mma_commit(&bars[SM::kAEmpty + ea]);
         sm100::mma_commit(&bars[SM::kAccFull + ab]);
-        mma_issued = it + 1;
+        used = true;
+        ++mma_issued;
       }
     }
-  } else if (BULK && lane == 0) {
-    // ------------------------------------------------------------ raw key rows
-    for (; issued < n_it; ++issued) {
-      const int j = (int)issued, slot = j % kStages;
-      if (j >= kStages && !wait(SM::kEmpty + slot, (uint32_t)((j / kStages - 1) & 1), 28)) break;
-      const int64_t t = t0 + j, g = t / tpg, kin0 = (t % tpg) * 128;
-      const int64_t key0 = g * p.kpg + p.key_base + kin0;
-      const int64_t left = p.nkeys - kin0;
-      const int rows = left < 128 ? (int)left : 128;
-      uint8_t *st = sStage + slot * SM::kStageBytes;
-      const uint32_t cb = rows * CW * 4, sb = rows * NG * 4;
-      sm100::mbar_expect_tx(&bars[SM::kFull + slot], cb + sb);
-      sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
-      sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
+  } else if (lane == 0) {
+    // ------------------------------------------------------------ copies
+    TileWalk tw(t0, tpg);
+    for (; issued < n_it; ++issued, tw.advance(1)) {
+      const int j = (int)(tw.g - g0);
+      if (j == b_loaded) {  // first tile of a group: its query operand
+        if (j >= 2 && !wait(SM::kBEmpty + (j & 1), (uint32_t)(((j >> 1) - 1) & 1), 30)) break;
+        sm100::mbar_expect_tx(&bars[SM::kBFull + (j & 1)], b_bytes);
+        sm100::bulk_load(sB + (j & 1) * b_bytes, p.qop + tw.g * (int64_t)b_bytes, b_bytes, &bars[SM::kBFull + (j & 1)]);
+        ++b_loaded;
+      }
+      if constexpr (BULK) {
+        const int jt = (int)issued, slot = jt % kStages;
+        if (jt >= kStages && !wait(SM::kEmpty + slot, (uint32_t)((jt / kStages - 1) & 1), 28)) break;
+        const int64_t kin0 = tw.tin * 128;
+        const int64_t key0 = tw.g * p.kpg + p.key_base + kin0;
+        const int64_t left = p.nkeys - kin0;
+        const int rows = left < 128 ? (int)left : 128;
+        uint8_t *st = sStage + slot * SM::kStageBytes;
+        const uint32_t cb = rows * CW * 4, sb = rows * NG * 4;
+        sm100::mbar_expect_tx(&bars[SM::kFull + slot], cb + sb);
+        sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
+        sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
+      }
     }
   }
   // ------------------------------------------------------------ teardown
   __syncthreads();
-  if (warp == kMmaWarp && lane == 0) {
-    if (mma_issued > 0) {  // no MMA may still write TMEM when it is freed
-      sm100::mma_commit(&bars[SM::kMmaDone]);
-      sm100::mbar_wait(&bars[SM::kMmaDone], md_ph, p.err, 29);
-    }
-    if (b_pending) sm100::mbar_wait(&bars[SM::kBFull], b_ph, p.err, 30);
+  if (warp >= kMmaWarp && warp < kLoadWarp && lane == 0 && mma_issued > 0) {
+    // no MMA may still write TMEM when it is freed
+    sm100::mma_commit(&bars[SM::kMmaDone + (warp - kMmaWarp)]);
+    sm100::mbar_wait(&bars[SM::kMmaDone + (warp - kMmaWarp)], 0u, p.err, 29);
   }
-  if (BULK && warp == kLoadWarp && lane == 0 && *sAbort) {
-    // copies issued but possibly not consumed: the last kStages issued
-    for (int64_t j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-      sm100::mbar_wait(&bars[SM::kFull + j % kStages], (uint32_t)((j / kStages) & 1), p.err, 31);
+  if (warp == kLoadWarp && lane == 0 && *sAbort) {
+    // copies issued but possibly not consumed: the last kStages key stages
+    // and the last two query operands
+    if constexpr (BULK) {
+      for (int64_t j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+        sm100::mbar_wait(&bars[SM::kFull + j % kStages], (uint32_t)((j / kStages) & 1), p.err, 31);
+    }
+    for (int j = b_loaded > 2 ? b_loaded - 2 : 0; j < b_loaded; ++j)
+      sm100::mbar_wait(&bars[SM::kBFull + (j & 1)], (uint32_t)((j >> 1) & 1), p.err, 32);
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -520,7 +614,7 @@ tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, in
   const bool bulk = ng == 4 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
                     reinterpret_cast<uintptr_t>(signs) % 16 == 0;
   if (reinterpret_cast<uintptr_t>(qop) % 16 != 0) return TQ_ERR_ALIGNMENT;
-  const size_t smem = 1024 + (bulk ? kStages * stage_bytes : 0) + (size_t)N * kScoreKBytes + 8 * 24 + 16;
+  const size_t smem = 1024 + (bulk ? kStages * stage_bytes : 0) + 2 * (size_t)N * kScoreKBytes + 8 * 48 + 16;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -61,6 +61,7 @@ constexpr uint32_t kWaitSlices = 2000;      // about 2 s in all
 // Bounded wait; on timeout writes `code` to *err (if not yet set) and
 // returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code) {
+  if (mbar_try_wait(bar, parity)) return true;  // already complete: no sleep
   for (uint32_t i = 0; i < kWaitSlices; ++i)
     if (mbar_try_wait_for(bar, parity, kWaitSliceNs)) return true;
   atomicCAS(err, 0, code);
@@ -71,6 +72,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
 // raised *abort; on its own timeout it records `code` and raises *abort.
 __device__ __forceinline__ bool mbar_wait_abort(uint64_t *bar, uint32_t parity, volatile int *abort, int *err,
                                                 int code) {
+  if (mbar_try_wait(bar, parity)) return true;
   for (uint32_t i = 0; i < kWaitSlices; ++i) {
     if (mbar_try_wait_for(bar, parity, kWaitSliceNs)) return true;
     if (*abort) return false;
