@@ -659,26 +659,31 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     return ~wbits;
   };
 
-  // thread 0's bookkeeping of loads in flight
+  // Two issuing threads in different warps: an issuing thread spends tens of
+  // cycles per tcgen05 instruction, so the rotation (thread kRotIssuer, with
+  // the x loads it waits for) and the QJL projection (thread 0) are split.
+  constexpr int kRotIssuer = 160;
+  // the rotation issuer's bookkeeping of loads in flight
   bool pend_full[2] = {false, false};
   uint32_t ph_full[2] = {0u, 0u};
   uint32_t ph_rot = 0u, ph_qjl = 0u;
-  bool failed = false;
+  bool failed = false;  // CTA-uniform: only ever set from a barrier vote
+  bool ifail = false;   // an issuing thread's own failed wait, voted at the next barrier
 
   // ---- prologue: tiles 0 and 1 loaded, rotation of tile 0, its norm parts
   if (nloc > 0) {
-    if (tid == 0) {
+    if (tid == kRotIssuer) {
       issue_tma(0, first);
       pend_full[0] = true;
       if (nloc > 1) {
         issue_tma(1, first + stride);
         pend_full[1] = true;
       }
-      failed = !sm100::mbar_wait(&bars[0], ph_full[0], p.err, 11);
+      ifail = !sm100::mbar_wait(&bars[0], ph_full[0], p.err, 11);
       ph_full[0] ^= 1u;
-      pend_full[0] = false;
+      pend_full[0] = ifail;
       sm100::tc_fence_after();
-      if (!failed) issue_rot(0, kColU0);
+      if (!ifail) issue_rot(0, kColU0);
     }
     bool ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 12);
     ph_rot ^= 1u;
@@ -686,19 +691,19 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     row_partial(kColU0, norm_col(0));
     sm100::tmem_wait_st();
     sm100::tc_fence_before();
-    failed = __syncthreads_or(!ok || failed) != 0;
+    failed = __syncthreads_or(!ok || ifail) != 0;
     sm100::tc_fence_after();
-    if (tid == 0 && !failed) {
+    if (tid == kRotIssuer && !failed) {
       if (nloc > 2) {
         issue_tma(0, first + 2 * stride);  // tile 0's rotation is done with buffer 0
         pend_full[0] = true;
       }
       if (nloc > 1) {
-        failed = !sm100::mbar_wait(&bars[1], ph_full[1], p.err, 13);
+        ifail = !sm100::mbar_wait(&bars[1], ph_full[1], p.err, 13);
         ph_full[1] ^= 1u;
-        pend_full[1] = false;
+        pend_full[1] = ifail;
         sm100::tc_fence_after();
-        if (!failed) issue_rot(1, 128u);
+        if (!ifail) issue_rot(1, 128u);
       }
     }
   }
@@ -709,7 +714,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   const float2 half2v = make_float2(0.5f, 0.5f);
   const float2 base2 = make_float2(8388608.0f + (float)(HALF - 1), 8388608.0f + (float)(HALF - 1));
   int it = 0;
-  for (; it < nloc && !failed; ++it) {
+  for (; it < nloc && !failed; ++it) {  // `failed` is CTA-uniform
     const int t = first + it * stride;
     const int par = it & 1;
     const uint32_t ucol = par ? 128u : 0u;
@@ -793,22 +798,22 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tmem_wait_st();
     sm100::fence_proxy_async();
     sm100::tc_fence_before();
-    failed = __syncthreads_or(!ok || failed) != 0;
+    failed = __syncthreads_or(!ok || ifail) != 0;
     if (failed) break;
     sm100::tc_fence_after();
     // ---- (e) QJL projection of this tile; the rotation two tiles ahead
-    if (tid == 0) {
-      issue_qjl();
+    if (tid == 0) issue_qjl();
+    if (tid == kRotIssuer) {
       if (it + 3 < nloc) {  // tile it+1's rotation is done with its buffer
         issue_tma(par ^ 1, first + (it + 3) * stride);
         pend_full[par ^ 1] = true;
       }
       if (it + 2 < nloc) {
-        failed = !sm100::mbar_wait(&bars[par], ph_full[par], p.err, 17);
+        ifail = !sm100::mbar_wait(&bars[par], ph_full[par], p.err, 17);
         ph_full[par] ^= 1u;
-        pend_full[par] = false;
+        pend_full[par] = ifail;
         sm100::tc_fence_after();
-        if (!failed) issue_rot(par, ucol);  // U of this tile has been read
+        if (!ifail) issue_rot(par, ucol);  // U of this tile has been read
       }
     }
     prev_norm = nrm;
@@ -816,6 +821,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   }
 
   // ---- drain: sign bits and norms of the last tile
+  failed = __syncthreads_or(failed || ifail) != 0;
   if (!failed && it > 0) {
     const bool ok = __syncthreads_and(sm100::mbar_wait(&bars[3], ph_qjl, p.err, 18)) != 0;  // CTA-uniform
     sm100::tc_fence_after();
@@ -828,9 +834,14 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       }
     }
   }
-  if (failed && tid == 0) {
+  if (failed && tid == kRotIssuer) {
     for (int b = 0; b < 2; ++b)
       if (pend_full[b]) sm100::mbar_wait(&bars[b], ph_full[b], p.err, 16);
+  }
+  if (failed && (tid == 0 || tid == kRotIssuer)) {
+    // MMAs this thread issued may still run: wait (bounded) before TMEM is freed
+    sm100::mma_commit(&bars[tid == 0 ? 3 : 2]);
+    sm100::mbar_wait(&bars[tid == 0 ? 3 : 2], tid == 0 ? ph_qjl : ph_rot, p.err, 19);
   }
   sm100::tc_fence_before();
   __syncthreads();
