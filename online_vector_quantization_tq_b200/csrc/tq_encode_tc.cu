@@ -536,7 +536,7 @@ struct Enc2Smem {
 }  // namespace
 
 template <int D, int W>
-__global__ void __launch_bounds__(128 * (D / 32), 1)
+__global__ void __launch_bounds__(128 * (D / 32) + 32, 1)
 k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   constexpr int P = D / 32;
   constexpr int L = 1 << W;
@@ -550,16 +550,21 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   uint8_t *sAr = smem + SM::kOffAr;
   uint8_t *sBr = smem + SM::kOffBr;
   uint8_t *sBs = smem + SM::kOffBs;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffMisc);  // full[2], rot, qjl
-  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffMisc);  // full[2], rot, qjl, drain
+  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 5);
 
   const int tid = threadIdx.x;
   const int row = tid & (kRows - 1);
   const int pc = tid >> 7;  // column group
   const uint32_t lane = (uint32_t)(row & ~31) << 16;
+  // warps 0 .. 4P-1 compute; the last warp only issues copies and MMAs (an
+  // issuing thread spends tens of cycles per tcgen05 instruction, which
+  // would otherwise hold up a computing warp and, at the tile barrier, all)
+  constexpr int kIssuer = 128 * P;
+  const bool compute = tid < kIssuer;
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) sm100::mbar_init(&bars[i], 1);
+    for (int i = 0; i < 5; ++i) sm100::mbar_init(&bars[i], 1);
     sm100::fence_barrier_init();
     sm100::prefetch_tmap(&xmap);
   }
@@ -659,11 +664,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     return ~wbits;
   };
 
-  // Two issuing threads in different warps: an issuing thread spends tens of
-  // cycles per tcgen05 instruction, so the rotation (thread kRotIssuer, with
-  // the x loads it waits for) and the QJL projection (thread 0) are split.
-  constexpr int kRotIssuer = 160;
-  // the rotation issuer's bookkeeping of loads in flight
+  // the issuer's bookkeeping of loads in flight
   bool pend_full[2] = {false, false};
   uint32_t ph_full[2] = {0u, 0u};
   uint32_t ph_rot = 0u, ph_qjl = 0u;
@@ -672,7 +673,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
 
   // ---- prologue: tiles 0 and 1 loaded, rotation of tile 0, its norm parts
   if (nloc > 0) {
-    if (tid == kRotIssuer) {
+    if (tid == kIssuer) {
       issue_tma(0, first);
       pend_full[0] = true;
       if (nloc > 1) {
@@ -685,15 +686,18 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       sm100::tc_fence_after();
       if (!ifail) issue_rot(0, kColU0);
     }
-    bool ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 12);
-    ph_rot ^= 1u;
-    sm100::tc_fence_after();
-    row_partial(kColU0, norm_col(0));
-    sm100::tmem_wait_st();
+    bool ok = true;
+    if (compute) {
+      ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 12);
+      ph_rot ^= 1u;
+      sm100::tc_fence_after();
+      row_partial(kColU0, norm_col(0));
+      sm100::tmem_wait_st();
+    }
     sm100::tc_fence_before();
     failed = __syncthreads_or(!ok || ifail) != 0;
     sm100::tc_fence_after();
-    if (tid == kRotIssuer && !failed) {
+    if (tid == kIssuer && !failed) {
       if (nloc > 2) {
         issue_tma(0, first + 2 * stride);  // tile 0's rotation is done with buffer 0
         pend_full[0] = true;
@@ -720,6 +724,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     const uint32_t ucol = par ? 128u : 0u;
     const int64_t grow = (int64_t)t * kRows + row;
     bool ok = true;
+    if (compute) {
     // ---- (a) this tile's rotated row (its MMA completed before the last barrier)
     const float nacc = sqrtf(sum_parts(norm_col(par)));
     const float nrm = nacc * p.rho;
@@ -797,13 +802,16 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tmem_st1(tmem + lane + gam_col(par) + pc, __float_as_uint(g2.x + g2.y));
     sm100::tmem_wait_st();
     sm100::fence_proxy_async();
+    prev_norm = nrm;
+    prev_row = grow;
+    }  // compute
     sm100::tc_fence_before();
     failed = __syncthreads_or(!ok || ifail) != 0;
     if (failed) break;
     sm100::tc_fence_after();
     // ---- (e) QJL projection of this tile; the rotation two tiles ahead
-    if (tid == 0) issue_qjl();
-    if (tid == kRotIssuer) {
+    if (tid == kIssuer) {
+      issue_qjl();
       if (it + 3 < nloc) {  // tile it+1's rotation is done with its buffer
         issue_tma(par ^ 1, first + (it + 3) * stride);
         pend_full[par ^ 1] = true;
@@ -816,16 +824,14 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         if (!ifail) issue_rot(par, ucol);  // U of this tile has been read
       }
     }
-    prev_norm = nrm;
-    prev_row = grow;
   }
 
   // ---- drain: sign bits and norms of the last tile
   failed = __syncthreads_or(failed || ifail) != 0;
   if (!failed && it > 0) {
-    const bool ok = __syncthreads_and(sm100::mbar_wait(&bars[3], ph_qjl, p.err, 18)) != 0;  // CTA-uniform
+    const bool ok = __syncthreads_and(compute ? sm100::mbar_wait(&bars[3], ph_qjl, p.err, 18) : true) != 0;
     sm100::tc_fence_after();
-    if (ok) {
+    if (ok && compute) {
       const uint32_t sw = sign_word();
       const float gam = pc == 0 ? sqrtf(sum_parts(gam_col((it - 1) & 1))) * (1.0f / kRScale) : 0.f;
       if (prev_row >= 0 && prev_row < p.n) {
@@ -834,14 +840,14 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       }
     }
   }
-  if (failed && tid == kRotIssuer) {
+  if (failed && tid == kIssuer) {
     for (int b = 0; b < 2; ++b)
       if (pend_full[b]) sm100::mbar_wait(&bars[b], ph_full[b], p.err, 16);
   }
-  if (failed && (tid == 0 || tid == kRotIssuer)) {
-    // MMAs this thread issued may still run: wait (bounded) before TMEM is freed
-    sm100::mma_commit(&bars[tid == 0 ? 3 : 2]);
-    sm100::mbar_wait(&bars[tid == 0 ? 3 : 2], tid == 0 ? ph_qjl : ph_rot, p.err, 19);
+  if (failed && tid == kIssuer) {
+    // MMAs issued may still run: wait (bounded) before TMEM is freed
+    sm100::mma_commit(&bars[4]);
+    sm100::mbar_wait(&bars[4], 0u, p.err, 19);
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -873,7 +879,7 @@ tq_status launch_tc2(const void *x, int64_t n, int64_t ldx, const EncTCParams &p
   auto kern = k_encode_tc2<D, W>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TQ_ERR_CUDA;
-  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32), smem, st>>>(map, pp);
+  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32) + 32, smem, st>>>(map, pp);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 }  // namespace
