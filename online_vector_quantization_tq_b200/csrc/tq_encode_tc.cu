@@ -522,6 +522,64 @@ namespace tq {
 // ============================================================================
 namespace {
 
+// Codes arrive as the bit patterns of the floats 2^23 + code.  Adding each
+// pattern shifted to the code's place and subtracting, per word, what the
+// 2^23 parts sum to (mod 2^32) leaves exactly the codes: one integer
+// multiply-add per code.  With W = 3 the codes of coordinates 24..31 are
+// spread over the fourth bit of every nibble; they are gathered as nibbles
+// first and distributed at the end.
+template <int W>
+__host__ __device__ constexpr uint32_t raw_offset(int word) {
+  uint32_t k = 0;
+  for (int i = 0; i < (W == 3 ? 24 : 32); ++i) {
+    const int p0 = code_bit_pos<W>(i, 0);
+    if ((p0 >> 5) == word) k += 0x4B000000u << (p0 & 31);
+  }
+  return k;
+}
+__host__ __device__ constexpr uint32_t raw_tail_offset() {
+  uint32_t k = 0;
+  for (int i = 0; i < 8; ++i) k += 0x4B000000u << (4 * i);
+  return k;
+}
+
+template <int W>
+struct RawPack {
+  uint32_t w[W], tail;
+  __device__ __forceinline__ RawPack() : tail(0u) {
+#pragma unroll
+    for (int k = 0; k < W; ++k) w[k] = 0u;
+  }
+  __device__ __forceinline__ void add(int i, uint32_t raw) {  // i: coordinate in the group (unrolled)
+    if (W == 3 && i >= 24) {
+      tail += raw << (4 * (i - 24));
+    } else {
+      const int p0 = code_bit_pos<W>(i, 0);
+      w[p0 >> 5] += raw << (p0 & 31);
+    }
+  }
+  __device__ __forceinline__ void finish(uint32_t (&out)[W]) const {
+#pragma unroll
+    for (int k = 0; k < W; ++k) out[k] = w[k] - raw_offset<W>(k);
+    if constexpr (W == 3) {
+      const uint32_t t = tail - raw_tail_offset();
+      out[0] |= (t & 0x44444444u) << 1;
+      out[1] |= (t & 0x22222222u) << 2;
+      out[2] |= (t & 0x11111111u) << 3;
+    }
+  }
+};
+
+// d = a * b + c on two lanes, rounded down
+__device__ __forceinline__ float2 ffma2_rm(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rm.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
+        "l"(*reinterpret_cast<const uint64_t *>(&c)));
+  return *reinterpret_cast<const float2 *>(&r);
+}
+
 template <int D>
 struct Enc2Smem {
   static constexpr int kXBytes = kRows * D * 2;
@@ -536,7 +594,7 @@ struct Enc2Smem {
 }  // namespace
 
 template <int D, int W>
-__global__ void __launch_bounds__(128 * (D / 32) + 32, 1)
+__global__ void __launch_bounds__(128 * (D / 32), 1)
 k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   constexpr int P = D / 32;
   constexpr int L = 1 << W;
@@ -557,14 +615,15 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   const int row = tid & (kRows - 1);
   const int pc = tid >> 7;  // column group
   const uint32_t lane = (uint32_t)(row & ~31) << 16;
-  // warps 0 .. 4P-1 compute; the last warp only issues copies and MMAs (an
-  // issuing thread spends tens of cycles per tcgen05 instruction, which
-  // would otherwise hold up a computing warp and, at the tile barrier, all)
-  constexpr int kIssuer = 128 * P;
-  const bool compute = tid < kIssuer;
+  // Two issuing threads in different warps: an issuing thread spends tens of
+  // cycles per tcgen05 instruction, so the rotation (thread kIssuer, with the
+  // x loads it waits for) and the QJL projection (thread 0) are split.
+  constexpr int kIssuer = 160;
+  constexpr bool compute = true;
 
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) sm100::mbar_init(&bars[i], 1);
+    for (int i = 0; i < 4; ++i) sm100::mbar_init(&bars[i], 1);
+    sm100::mbar_init(&bars[4], 2);  // failure drain: both issuing threads commit
     sm100::fence_barrier_init();
     sm100::prefetch_tmap(&xmap);
   }
@@ -587,12 +646,12 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   // 2^-40, so the step is exactly 0 or 1 (u^2 vs the rounded T_k^2 can only
   // disagree with |u| vs T_k within an ulp of the threshold).
   constexpr float kBig = 1099511627776.0f;  // 2^40
-  float nT2B[HALF], dC[HALF];
+  float nT2B[HALF], ndC[HALF];  // -T_k^2 2^40, minus the centroid steps
 #pragma unroll
   for (int k = 0; k < HALF; ++k) {
     const float tk = p.thr_s[HALF - 1 + k];
     nT2B[k] = -(tk * tk) * kBig;
-    dC[k] = k == 0 ? p.cen_s[HALF] : p.cen_s[HALF + k] - p.cen_s[HALF + k - 1];
+    ndC[k] = -(k == 0 ? p.cen_s[HALF] : p.cen_s[HALF + k] - p.cen_s[HALF + k - 1]);
   }
 
   const uint32_t idesc_rot = sm100::idesc_bf16_f32(kRows, D);
@@ -715,8 +774,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   float prev_norm = 0.f;
   int64_t prev_row = -1;
   const float2 big2 = make_float2(kBig, kBig);
-  const float2 half2v = make_float2(0.5f, 0.5f);
-  const float2 base2 = make_float2(8388608.0f + (float)(HALF - 1), 8388608.0f + (float)(HALF - 1));
+  const float2 base2 = make_float2(8388608.0f + (float)HALF, 8388608.0f + (float)HALF);
   int it = 0;
   for (; it < nloc && !failed; ++it) {  // `failed` is CTA-uniform
     const int t = first + it * stride;
@@ -733,32 +791,32 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     uint32_t acc[32];
     sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
     sm100::tmem_wait_ld();
-    uint32_t cw[W];
-#pragma unroll
-    for (int k = 0; k < W; ++k) cw[k] = 0u;
+    RawPack<W> pk;
     uint32_t hi[16], lo[16];
     float2 g2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
       const float2 us = __fmul2_rn(make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])), sv2);
       const float2 usb = __fmul2_rn(us, big2);
-      float2 cm = make_float2(dC[0], dC[0]), m = make_float2(0.f, 0.f);
+      // m + 1/2 (m = thresholds passed by |u|) and -c[code] magnitude
+      float2 ncm = make_float2(ndC[0], ndC[0]), mh = make_float2(0.5f, 0.5f);
 #pragma unroll
       for (int k = 1; k < HALF; ++k) {
         const float2 st = make_float2(__saturatef(__fmaf_rn(us.x, usb.x, nT2B[k])),
                                       __saturatef(__fmaf_rn(us.y, usb.y, nT2B[k])));
-        cm = __ffma2_rn(st, make_float2(dC[k], dC[k]), cm);
-        m = __fadd2_rn(m, st);
+        ncm = __ffma2_rn(st, make_float2(ndC[k], ndC[k]), ncm);
+        mh = __fadd2_rn(mh, st);
       }
-      // s = +-1 from the sign bit (u = -0 takes the lower middle code)
-      const uint32_t bx = __float_as_uint(us.x) & 0x80000000u, by = __float_as_uint(us.y) & 0x80000000u;
-      const float2 sg = make_float2(__uint_as_float(bx | 0x3F800000u), __uint_as_float(by | 0x3F800000u));
-      const float2 nsg = make_float2(__uint_as_float(bx ^ 0xBF800000u), __uint_as_float(by ^ 0xBF800000u));
-      const float2 cb = __fadd2_rn(__ffma2_rn(sg, half2v, half2v), base2);
-      const float2 codef = __ffma2_rn(sg, m, cb);  // 2^23 + code
-      const float2 rr = __ffma2_rn(nsg, cm, us);   // u - c[code]
-      pack_code<W>(cw, j, __float_as_uint(codef.x) & (uint32_t)(L - 1));
-      pack_code<W>(cw, j + 1, __float_as_uint(codef.y) & (uint32_t)(L - 1));
+      // s = +-1 from the sign bit (u = -0 takes the lower middle code); the
+      // code is HALF - 1/2 + s (m + 1/2): 2^23 + HALF + s (m + 1/2) is
+      // exactly 2^23 + code + 1/2 (never below 2^23), rounded down to
+      // 2^23 + code
+      const float2 sg = make_float2(__uint_as_float((__float_as_uint(us.x) & 0x80000000u) | 0x3F800000u),
+                                    __uint_as_float((__float_as_uint(us.y) & 0x80000000u) | 0x3F800000u));
+      const float2 codef = ffma2_rm(sg, mh, base2);
+      const float2 rr = __ffma2_rn(sg, ncm, us);  // u - c[code]
+      pk.add(j, __float_as_uint(codef.x));
+      pk.add(j + 1, __float_as_uint(codef.y));
       g2 = __ffma2_rn(rr, rr, g2);
       const __half2 h = __floats2half2_rn(rr.x, rr.y);
       const float2 hf = __half22float2(h);
@@ -766,6 +824,8 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       const float2 lf = __fadd2_rn(rr, make_float2(-hf.x, -hf.y));
       lo[j / 2] = pack_half2(lf.x, lf.y);
     }
+    uint32_t cw[W];
+    pk.finish(cw);
     if (grow < p.n) {
       uint32_t *dst = p.codes + grow * p.out_stride * (W * D / 32) + pc * W;
 #pragma unroll
@@ -810,8 +870,8 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     if (failed) break;
     sm100::tc_fence_after();
     // ---- (e) QJL projection of this tile; the rotation two tiles ahead
+    if (tid == 0) issue_qjl();
     if (tid == kIssuer) {
-      issue_qjl();
       if (it + 3 < nloc) {  // tile it+1's rotation is done with its buffer
         issue_tma(par ^ 1, first + (it + 3) * stride);
         pend_full[par ^ 1] = true;
@@ -844,7 +904,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     for (int b = 0; b < 2; ++b)
       if (pend_full[b]) sm100::mbar_wait(&bars[b], ph_full[b], p.err, 16);
   }
-  if (failed && tid == kIssuer) {
+  if (failed && (tid == 0 || tid == kIssuer)) {
     // MMAs issued may still run: wait (bounded) before TMEM is freed
     sm100::mma_commit(&bars[4]);
     sm100::mbar_wait(&bars[4], 0u, p.err, 19);
@@ -879,7 +939,7 @@ tq_status launch_tc2(const void *x, int64_t n, int64_t ldx, const EncTCParams &p
   auto kern = k_encode_tc2<D, W>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TQ_ERR_CUDA;
-  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32) + 32, smem, st>>>(map, pp);
+  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32), smem, st>>>(map, pp);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 }  // namespace
