@@ -35,6 +35,11 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 
 METRIC = "keys scored/s and vectors encoded/s (1 B200), as % of HBM roofline"
+# DRAM bytes (read + write) of one launch on the kv workload, from the ncu
+# captures summarised in profiles/encode_tc2_kv.md and profiles/score_tc_kv.md;
+# set to None whenever the kernel changes after its capture.
+ENCODE_TRAFFIC_BYTES = 324954624
+SCORE_TRAFFIC_BYTES = 79327232
 
 
 def _peaks():
@@ -51,7 +56,9 @@ class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a region.
 
     Samples every GPU the driver shows and keeps the one whose UUID matches
-    the CUDA device (or the only one, when just one is visible)."""
+    the CUDA device (or the only one, when just one is visible).  A reader
+    thread collects the lines as they come, so the caller can keep the GPU
+    under load until samples have arrived."""
 
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -60,33 +67,50 @@ class ClockSampler:
     def __init__(self, uuid: str):
         self.uuid = (uuid or "").lower().replace("gpu-", "")
         self.proc = None
-        self.out = None
+        self.lines = []
         self.error = None
+        self.thread = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln)
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
         except Exception as e:  # no nvidia-smi
             self.error = str(e)
             self.proc = None
         return self
 
+    def count(self) -> int:
+        return len(self.lines)
+
+    def wait_first(self, timeout: float = 20.0):
+        t_end = time.time() + timeout
+        while self.proc is not None and not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.05)
+
     def __exit__(self, *exc):
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, err = self.proc.communicate(timeout=5)
-                if not self.out:
+                _, err = self.proc.communicate(timeout=5)
+                if not self.lines:
                     self.error = (err or "").strip()[:200]
             except Exception:
                 self.proc.kill()
-                self.out = ""
+            if self.thread is not None:
+                self.thread.join(timeout=5)
 
     def summary(self):
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lines = [[x.strip() for x in ln.split(",")] for ln in (self.out or "").strip().splitlines()]
+        lines = [[x.strip() for x in ln.split(",")] for ln in self.lines if ln.strip()]
         lines = [ln for ln in lines if len(ln) >= 8]
         uuids = sorted({ln[0].lower().replace("gpu-", "") for ln in lines})
         if self.uuid in uuids:
@@ -167,12 +191,14 @@ def run_tq(args, rank, world, local):
     props = torch.cuda.get_device_properties(dev)
     recs = []
     with ClockSampler(str(getattr(props, "uuid", ""))) as clk:
-        # keep the GPU busy for ~1 s before the timed steps so the clock
-        # samples (every 100 ms) cover the load
-        pre = max(1, int(1.0 / max(warm_ms * 1e-3, 1e-5)))
-        for _ in range(pre):
-            step()
-        torch.cuda.synchronize(dev)
+        # the same load before (until three samples came in, at most ~3 s)
+        # and after the timed steps, so the 100 ms clock samples cover it
+        clk.wait_first()
+        n0, t_end = clk.count(), time.time() + 3.0
+        while clk.count() < n0 + 3 and time.time() < t_end:
+            for _ in range(max(1, int(0.05 / max(warm_ms * 1e-3, 1e-5)))):
+                step()
+            torch.cuda.synchronize(dev)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -182,6 +208,11 @@ def run_tq(args, rank, world, local):
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
+        n1, t_end = clk.count(), time.time() + 1.0
+        while clk.count() < n1 + 2 and time.time() < t_end:
+            for _ in range(max(1, int(0.05 / max(warm_ms * 1e-3, 1e-5)))):
+                step()
+            torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1) / args.steps
     enc_ms = statistics.mean(a.elapsed_time(b_) for a, b_, _ in recs)
     score_ms = statistics.mean(b_.elapsed_time(c) for _, b_, c in recs)
@@ -251,10 +282,13 @@ def run_tq(args, rank, world, local):
             "encode_ms": enc_ms,
             "score_ms": score_ms,
             "roofline": {"bound": "hbm", "kernel": "encode", "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": ENCODE_TRAFFIC_BYTES,
                          "algorithmic_bytes_per_launch": enc_bytes},
             "score_roofline": {"bound": "hbm", "achieved": score_bytes / (score_ms * 1e-3) / 1e9, "peak": peak,
-                               "unit": "GB/s", "frac": score_bytes / (score_ms * 1e-3) / 1e9 / peak},
+                               "unit": "GB/s", "frac": score_bytes / (score_ms * 1e-3) / 1e9 / peak,
+                               "traffic": SCORE_TRAFFIC_BYTES,
+                               "note": "phase time: query preparation kernels + the scorer"},
             "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "keys/s",
                     "h2d_bytes_per_step": x_pin.numel() * 2 + y_pin.numel() * 4,
                     "d2h_bytes_per_step": out_pin.numel() * 4},
