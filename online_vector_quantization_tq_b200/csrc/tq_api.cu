@@ -58,6 +58,7 @@ extern "C" {
 
 size_t tq_encode_workspace_bytes(const tq_quantizer *q, int64_t n) {
   if (!q || n <= 0 || fwht_fast(q)) return 0;
+  if (q->device >= 0 && dense_tc_supported(q)) return round_up(dense_tc_ws_bytes(q, n), 256);
   return round_up(v1_dense_ws_bytes(q, n), 256);
 }
 
@@ -78,8 +79,10 @@ tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype, int
   if (tc_encode_supported(q, dtype, ldx, chan != nullptr))
     return tc_encode(q, x, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, s);
   if (fwht_fast(q)) return v1_encode_fwht(q, src, n, codes, signs, norms, out_stride, s);
-  if (!workspace || !aligned(workspace, 16) || v1_dense_batch_rows(q, workspace_bytes) < 1)
-    return TQ_ERR_WORKSPACE;
+  if (!workspace || !aligned(workspace, 16)) return TQ_ERR_WORKSPACE;
+  if (dense_tc_supported(q))
+    return dense_tc_encode(q, src, n, codes, signs, norms, out_stride, workspace, workspace_bytes, s);
+  if (v1_dense_batch_rows(q, workspace_bytes) < 1) return TQ_ERR_WORKSPACE;
   return v1_encode_dense(q, src, n, codes, signs, norms, out_stride, workspace, workspace_bytes, s);
 }
 

@@ -381,8 +381,6 @@ k_encode_tc(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
 }
 
 // ------------------------------------------------------------------ host side
-namespace {
-
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -394,6 +392,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   }
   return fn;
 }
+
+namespace {
 
 template <int D, int W, int RP, int SRCW, bool GATHER>
 tq_status launch_tc(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, int64_t cols,

@@ -251,7 +251,35 @@ tq_status upload(T **dst, const T *src, size_t count) {
   return TQ_OK;
 }
 
+// v as 31-bit fixed point under one power-of-two scale 2^e (|v| 2^e < 2^30),
+// split into four signed-byte planes: round(v 2^e) = 2^24 a + 2^16 b +
+// 2^8 c + d with b, c, d in [-128, 127] and |a| <= 64.
+std::vector<int8_t> limb_split(const std::vector<double> &v, int *e_out) {
+  double big = 0.0;
+  for (double x : v) big = std::max(big, std::fabs(x));
+  int E = 0;
+  std::frexp(big, &E);  // big < 2^E
+  const int e = big > 0.0 ? 30 - E : 0;
+  const size_t n = v.size();
+  std::vector<int8_t> out(4 * n);
+  for (size_t i = 0; i < n; ++i) {
+    long t = std::lrint(std::ldexp(v[i], e));
+    for (int l = 3; l >= 1; --l) {  // low limbs, balanced
+      const long lo = ((t + 128) & 255) - 128;
+      out[(size_t)l * n + i] = (int8_t)lo;
+      t = (t - lo) / 256;
+    }
+    out[i] = (int8_t)t;
+  }
+  *e_out = e;
+  return out;
+}
+
 void free_device(tq_quantizer *q) {
+  cudaFree(q->d_rot_limbs);
+  cudaFree(q->d_qjl_limbs);
+  q->d_rot_limbs = nullptr;
+  q->d_qjl_limbs = nullptr;
   cudaFree(q->d_rot16);
   cudaFree(q->d_rot_bf16);
   cudaFree(q->d_err);
@@ -475,6 +503,19 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
       }
     }
     if (st == TQ_OK) st = upload(&q->d_rot16, pieces.data(), pieces.size());
+  }
+  if (st == TQ_OK && d >= 256) {
+    // fixed-point limbs of R and S for the dense tensor-core encode
+    const size_t dd = (size_t)d * d;
+    std::vector<double> rv(dd), sv((size_t)m * d);
+    for (size_t i = 0; i < dd; ++i) rv[i] = rot == TQ_ROT_HADAMARD ? q->rot_exact[i] : (double)q->rot[i];
+    for (size_t i = 0; i < sv.size(); ++i) sv[i] = half_bits_to_double(q->qjl16[i]);
+    const std::vector<int8_t> rl = limb_split(rv, &q->rot_limb_exp);
+    st = upload(&q->d_rot_limbs, rl.data(), rl.size());
+    if (st == TQ_OK) {
+      const std::vector<int8_t> sl = limb_split(sv, &q->qjl_limb_exp);
+      st = upload(&q->d_qjl_limbs, sl.data(), sl.size());
+    }
   }
   if (st == TQ_OK) {
     if (cudaMalloc((void **)&q->d_err, sizeof(int)) != cudaSuccess || cudaMemset(q->d_err, 0, sizeof(int)) != cudaSuccess) {

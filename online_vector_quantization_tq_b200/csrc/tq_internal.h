@@ -47,6 +47,13 @@ struct tq_quantizer {
   int tc_rot_pieces = 0;
   float tc_rho = 0.f;
   uint16_t *d_rot_bf16 = nullptr;  // Hadamard: d^1.5 R as two exact bf16 pieces [2][d][d]
+  // dense tensor-core encode (d >= 256): R and S as 31-bit fixed point,
+  // v 2^e = 2^24 a + 2^16 b + 2^8 c + d with signed bytes, stored as four
+  // planes [4][rows][d] (a, b, c, d)
+  int8_t *d_rot_limbs = nullptr;
+  int rot_limb_exp = 0;
+  int8_t *d_qjl_limbs = nullptr;
+  int qjl_limb_exp = 0;
   int *d_err = nullptr;          // device error word (bounded waits that timed out)
   // integer scorer: centroid c_k ~ (256 * ch[k] + cl[k]) * 2^-score_cexp
   int8_t score_ch[tq::kMaxLevels] = {}, score_cl[tq::kMaxLevels] = {};

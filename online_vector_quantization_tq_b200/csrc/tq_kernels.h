@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "tq_common.cuh"
 
@@ -25,6 +26,16 @@ tq_status v1_topk_select(float *score, const int64_t *idx, int64_t rows, int64_t
                          int64_t out_row_stride, cudaStream_t st);
 tq_status v1_sumsq(const RowSource &src, int64_t groups, int64_t rows_per_group, double *part, int nchunks,
                    double *out, cudaStream_t st);
+
+// cuTensorMapEncodeTiled from the driver (null if unavailable)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Dense rotation (any d that is a multiple of 64, from 256 up) on the tensor
+// cores: both projections as fp16-piece GEMMs with fused epilogues.
+bool dense_tc_supported(const tq_quantizer *q);
+size_t dense_tc_ws_bytes(const tq_quantizer *q, int64_t n);
+tq_status dense_tc_encode(const tq_quantizer *q, const RowSource &src, int64_t n, void *codes, void *signs,
+                          float *norms, int64_t out_stride, void *ws, size_t ws_bytes, cudaStream_t st);
 
 bool tc_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather);
 tq_status tc_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,

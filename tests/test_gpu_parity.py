@@ -225,6 +225,35 @@ def test_other_shapes(tq, d, b, rot):
                  d, rep.skip_rows)
 
 
+@pytest.mark.parametrize("d,b,rot", [(384, 3, "haar"), (512, 5, "hadamard"), (320, 4, "haar")])
+def test_dense_tensor_core_batches(tq, d, b, rot):
+    """Dense rotation on the tensor cores (fp16-piece GEMMs), forced through several
+    workspace batches: 1000 rows in batches of 256 (a ragged last batch), a zero row,
+    and a partial 256-column tile when d is not a multiple of 256."""
+    rng = np.random.default_rng(d * 7 + b)
+    n = 1000
+    x = (rng.standard_normal((n, d)) * 3.0).astype(np.float32)
+    x[17] = 0.0
+    t = tables(d, b, rot)
+    q = tq.tq_codebook(d, b, seed=0, rotation=rot)
+    nbytes = tq.lib().tq_encode_workspace_bytes(q.handle, 256)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    enc = tq.tq_encode(q, dev(x), workspace=ws)
+    rep = check_encode(*host(enc), x, t)
+    assert enc.norms[17, 0].item() == 0.0 and enc.norms[17, 1].item() > 0.0
+    # a workspace too small for one 128-row batch is refused
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_encode(q, dev(x[:4]), workspace=torch.empty(4096, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == 6
+    y = rng.standard_normal((3, d)).astype(np.float32)
+    s = tq.tq_score(q, dev(y), 1, 3, enc, n).cpu().numpy()
+    assert np.all(s[:, 17] == 0.0)  # the zero key scores 0 (its relative error is undefined)
+    skip = rep.skip_rows.copy()
+    skip[17] = True
+    check_scores(s, o.score(*o.prepare_query(y, t), rep.ref, t), rep.ref["norm"], np.linalg.norm(y, axis=1),
+                 d, skip)
+
+
 def test_edge_cases(tq):
     t = tables(128, 3)
     q = tq.tq_codebook(128, 3, seed=0)
