@@ -52,6 +52,15 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+def _bf16_peak():
+    """Dense bf16 TFLOP/s measured on this machine (burst), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a region.
 
@@ -314,6 +323,7 @@ def run_workload(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     phases = {}
+    flops_ = {}
 
     def timed(name, fn):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -394,6 +404,9 @@ def run_workload(args):
         n_units, unit = n, "vectors/s"
         bytes_ = {"encode": n * (4 * d + q.code_bytes + q.sign_bytes + 8),
                   "topk": n * (q.code_bytes + q.sign_bytes + 8)}
+        # the rotation and the QJL projection, and one product per (query, key,
+        # coordinate of [y~ | p]): the dense contractions of the step
+        flops_ = {"encode": 2.0 * n * d * (d + d), "topk": 2.0 * nq * n * (d + d)}
         desc = f"ann: 1e6 x 1536 fp32 (std i^-0.5, L2-normalised), Haar, b=4; {nq} queries, top-10"
 
         def step():
@@ -414,11 +427,15 @@ def run_workload(args):
     torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1) / args.steps
     peak, peak_kind = _peaks()
+    bf16_peak = _bf16_peak()
     ph = {}
     for name, evs in phases.items():
         pm = statistics.mean(a.elapsed_time(b) for a, b in evs)
         gbs = bytes_[name] / (pm * 1e-3) / 1e9
         ph[name] = {"ms": pm, "algorithmic_GBps": gbs, "frac_of_measured_hbm": gbs / peak}
+        if name in flops_:
+            tf = flops_[name] / (pm * 1e-3) / 1e12
+            ph[name].update({"algorithmic_TFLOPs": tf, "frac_of_measured_bf16": tf / bf16_peak})
     line = {"metric": METRIC, "value": n_units / (ms * 1e-3), "unit": unit, "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "data": "synthetic", "config": {"workload": desc}, "phases": ph,
@@ -493,7 +510,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", choices=["kv", "tiny", "kv_mixed", "decode", "ann"], default="kv")
-    ap.add_argument("--queries", type=int, default=16, help="ann workload: number of queries")
+    ap.add_argument("--queries", type=int, default=1024, help="ann workload: number of queries")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

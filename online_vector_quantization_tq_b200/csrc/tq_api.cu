@@ -127,7 +127,7 @@ tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq, 
 // Workspace of tq_score: prepared queries (y~, p), then the integer scorer's
 // query operand (at most 16 rows of 384 bytes per query) and per-query scales.
 struct ScoreLayout {
-  size_t ytil, p, qop, qsc, total;
+  size_t ytil, p, qop, qsc, dense, total;
 };
 ScoreLayout score_layout(const tq_quantizer *q, int64_t nq) {
   ScoreLayout L{};
@@ -140,6 +140,8 @@ ScoreLayout score_layout(const tq_quantizer *q, int64_t nq) {
   off += round_up((size_t)nq * 16 * 384, 256);
   L.qsc = off;
   off += round_up((size_t)nq * 16, 256);
+  L.dense = off;
+  if (dense_score_supported(q)) off += round_up(dense_score_ws_bytes(q, nq), 256);
   L.total = off;
   return L;
 }
@@ -177,6 +179,9 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_
     return tc_score(q, ytil, p, groups, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
                     keys_per_group, accumulate, reinterpret_cast<int8_t *>(ws + L.qop),
                     reinterpret_cast<float4 *>(ws + L.qsc), s);
+  if (dense_score_supported(q) && aligned(codes, 16) && aligned(signs, 16))
+    return dense_score(q, ytil, p, nq, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
+                       keys_per_group, accumulate, ws + L.dense, L.total - L.dense, s);
   return v1_score(q, ytil, p, nq, G, keys_per_group, 0, keys_per_group, codes, signs, norms, out,
                   keys_per_group, accumulate, s);
 }
@@ -188,7 +193,7 @@ constexpr int64_t kTopkChunk = 65536;
 constexpr int64_t kTopkSlice = 2048;
 
 struct TopkLayout {
-  size_t ytil, p, qop, qsc, scores, part_s, part_i, total;
+  size_t ytil, p, qop, qsc, scores, part_s, part_i, dense, total;
   int64_t chunk, nparts;
 };
 
@@ -211,6 +216,8 @@ TopkLayout topk_layout(const tq_quantizer *q, int64_t nq, int64_t n, int k) {
   off += round_up((size_t)nq * L.nparts * k * 4, 256);
   L.part_i = off;
   off += round_up((size_t)nq * L.nparts * k * 8, 256);
+  L.dense = off;
+  if (dense_score_supported(q)) off += round_up(dense_score_ws_bytes(q, nq), 256);
   L.total = off;
   return L;
 }
@@ -249,6 +256,7 @@ tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy
   st = v1_prepare_queries(q, src, nq, ytil, p, s);
   if (st != TQ_OK) return st;
   const bool tc = tc_score_supported(q, std::min<int64_t>(nq, 48)) && aligned(codes, 16) && aligned(signs, 16);
+  const bool dense = !tc && dense_score_supported(q) && aligned(codes, 16) && aligned(signs, 16);
   for (int64_t c0 = 0; c0 < n; c0 += L.chunk) {
     const int64_t cnt = std::min(L.chunk, n - c0);
     if (tc) {
@@ -259,6 +267,9 @@ tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy
                       reinterpret_cast<float4 *>(ws + L.qsc) + qb, s);
         if (st != TQ_OK) return st;
       }
+    } else if (dense) {
+      st = dense_score(q, ytil, p, nq, nq, n, c0, cnt, codes, signs, norms, scores, L.chunk, 0, ws + L.dense,
+                       L.total - L.dense, s);
     } else {
       st = v1_score(q, ytil, p, nq, nq, n, c0, cnt, codes, signs, norms, scores, L.chunk, 0, s);
     }

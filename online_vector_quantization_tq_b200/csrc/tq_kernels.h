@@ -37,6 +37,15 @@ size_t dense_tc_ws_bytes(const tq_quantizer *q, int64_t n);
 tq_status dense_tc_encode(const tq_quantizer *q, const RowSource &src, int64_t n, void *codes, void *signs,
                           float *norms, int64_t out_stride, void *ws, size_t ws_bytes, cudaStream_t st);
 
+// Scoring for d > 128 as an fp16 tensor-core GEMM over decoded keys (same
+// arguments and output as v1_score, plus its workspace).
+bool dense_score_supported(const tq_quantizer *q);
+size_t dense_score_ws_bytes(const tq_quantizer *q, int64_t nq);
+tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, int64_t nq_rows, int64_t G,
+                      int64_t kpg, int64_t key_base, int64_t nkeys, const void *codes, const void *signs,
+                      const float *norms, float *out, int64_t ldo, int accumulate, void *ws, size_t ws_bytes,
+                      cudaStream_t st);
+
 bool tc_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather);
 tq_status tc_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,
                     int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,
