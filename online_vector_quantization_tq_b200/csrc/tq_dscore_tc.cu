@@ -3,19 +3,23 @@
 // operands:
 //
 //   s(y, x) = ||x|| ( <y~, c[codes]> + gamma sqrt(pi/2)/m <p, 2 bits - 1> )
-//           = ||x|| < [y~ | kappa p], [c[codes] | gamma (2 bits - 1)] >,   kappa = sqrt(pi/2)/m
+//           = ||x|| < [y~ | y~ | kappa p], [c_hi | c_lo | gamma (2 bits - 1)] >
+//   with kappa = sqrt(pi/2)/m and c[codes] = c_hi + c_lo as two fp16 pieces.
 //
-//   k_dscore_queries  each query row [y~ | kappa p] scaled by a power of two
-//                     (largest entry below 2^14) as two fp16 pieces hi + lo;
-//   k_dscore_keys     a chunk of keys decoded to one fp16 row each (the codes'
-//                     centroids, then gamma (2 bit - 1));
-//   k_dscore_gemm     queries x keys, the two query pieces accumulated in
-//                     fp32 in TMEM; the epilogue scales by 2^-s and ||x|| and
-//                     writes the logits.
+//   k_dscore_queries  each query row [y~ | y~ | kappa p] scaled by a power of
+//                     two (largest entry below 2^14) as two fp16 pieces hi + lo;
+//   k_dscore_keys     a chunk of keys decoded to one fp16 row each;
+//   k_dscore_gemm     queries x keys: the high query piece against the whole
+//                     row, the low piece against all but c_lo (that product is
+//                     below 2^-22 of the score), fp32 accumulation in TMEM;
+//                     the epilogue scales by 2^-s and ||x|| and writes the
+//                     logits.
 //
-// Rounding the decoded key to fp16 moves a score by about 1.4e-4 of
-// ||x|| ||y|| / sqrt(d) (standard deviation, the rotation spreads the
-// coordinates evenly); the query pieces carry 22 bits.  Persistent CTAs walk
+// The centroids need the second piece: a single fp16 rounding of the table
+// is the same error for every coordinate holding that code, so it does not
+// average out over the dot product and reached 1.3e-3 of the score floor
+// ||x|| ||y|| / sqrt(d) in tests.  gamma in fp16 errs by at most 2^-12 of the
+// QJL term.  Persistent CTAs walk
 // 128-query x 256-key tiles with the queries of one key tile on consecutive
 // CTAs, so a key tile is read from HBM once and from L2 after that.
 #include <cudaTypedefs.h>
@@ -35,11 +39,12 @@ constexpr uint32_t kSStage = 2 * kSABytes + kSBBytes;  // query hi, query lo, ke
 constexpr int64_t kKeyChunk = 32768;
 
 struct DScoreParams {
-  int M, N, K;  // queries, keys, reduction (d + m)
+  int M, N, K;  // queries, keys, reduction (2d + m)
+  int d;
   int nstages;
   int *err;
   const float *qscale;  // [M] 2^-s of each query row
-  const float2 *norms;  // [N] the keys' (||x||, gamma), stride norm_stride
+  const float2 *norms;  // [N] the keys' (||x||, gamma)
   float *out;           // [M][ldo]
   int64_t ldo;
   int accumulate;
@@ -58,6 +63,7 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (p.M + kSBM - 1) / kSBM, ntk = (p.N + kSBN - 1) / kSBN;
   const int nitems = ntq * ntk, nk = (p.K + kSBK - 1) / kSBK;
+  const int lo_skip0 = p.d / kSBK, lo_skip1 = 2 * p.d / kSBK;  // K chunks of c_lo
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -132,7 +138,8 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
           sm100::tc_fence_after();
           const uint32_t sa = sm100::smem_u32(smem + slot * kSStage), sb = sa + 2 * kSABytes;
 #pragma unroll
-          for (int pc = 0; pc < 2; ++pc) {  // query hi, then query lo
+          for (int pc = 0; pc < 2; ++pc) {  // query hi, then query lo (not against c_lo)
+            if (pc == 1 && kc >= lo_skip0 && kc < lo_skip1) continue;
 #pragma unroll
             for (int ks = 0; ks < kSBK / 16; ++ks) {
               const uint64_t da = sm100::desc_sw128(sa + pc * kSABytes + ks * 32);
@@ -199,14 +206,16 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
   if (warp == 1) sm100::tmem_dealloc(tmem, 2 * kSBN);
 }
 
-// One warp per query row: [y~ | kappa p] 2^s as fp16 hi + lo.
+// One warp per query row: [y~ | y~ | kappa p] 2^s as fp16 hi + lo.
 __global__ void k_dscore_queries(const float *ytil, const float *p, int d, int m, int64_t nq, float kappa,
                                  __half *qh, __half *ql, float *qscale) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= nq) return;
-  const int K = d + m;
-  auto at = [&](int j) { return j < d ? ytil[row * d + j] : kappa * p[row * m + (j - d)]; };
+  const int K = 2 * d + m;
+  auto at = [&](int j) {
+    return j < 2 * d ? ytil[row * d + (j < d ? j : j - d)] : kappa * p[row * m + (j - 2 * d)];
+  };
   float big = 0.f;
   for (int j = lane; j < K; j += 32) big = fmaxf(big, fabsf(at(j)));
 #pragma unroll
@@ -223,27 +232,36 @@ __global__ void k_dscore_queries(const float *ytil, const float *p, int d, int m
   if (lane == 0) qscale[row] = ldexpf(1.0f, -s);
 }
 
-// One thread per (key, 32-coordinate group): the key's decoded row, fp16.
+// One thread per (key, 32-coordinate group of the row [c_hi | c_lo | gamma (2 bits - 1)]).
 template <int W>
 __global__ void k_dscore_keys(KernelTables kt, int64_t cnt, const uint32_t *codes, const uint32_t *signs,
                               const float2 *norms, __half *kop) {
-  const int ng = kt.d / 32, nsg = kt.m / 32, K = kt.d + kt.m;
+  const int ng = kt.d / 32, nsg = kt.m / 32, K = 2 * kt.d + kt.m, per = 2 * ng + nsg;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= cnt * (ng + nsg)) return;
-  const int64_t key = t / (ng + nsg);
-  const int grp = (int)(t % (ng + nsg));
+  if (t >= cnt * per) return;
+  const int64_t key = t / per;
+  const int grp = (int)(t % per);
   uint32_t hv[16];
-  if (grp < ng) {
+  if (grp < 2 * ng) {
+    const int cg = grp < ng ? grp : grp - ng;
+    const bool lo = grp >= ng;
     uint32_t w[W];
 #pragma unroll
-    for (int k = 0; k < W; ++k) w[k] = codes[key * (W * ng) + grp * W + k];
+    for (int k = 0; k < W; ++k) w[k] = codes[key * (W * ng) + cg * W + k];
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
-      const __half2 h = __floats2half2_rn(kt.centroids[unpack_code<W>(w, i)], kt.centroids[unpack_code<W>(w, i + 1)]);
+      float c2[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float c = kt.centroids[unpack_code<W>(w, i + h)];
+        const float chi = __half2float(__float2half_rn(c));
+        c2[h] = lo ? c - chi : chi;
+      }
+      const __half2 h = __floats2half2_rn(c2[0], c2[1]);
       hv[i / 2] = *reinterpret_cast<const uint32_t *>(&h);
     }
   } else {
-    const uint32_t sw = signs[key * nsg + (grp - ng)];
+    const uint32_t sw = signs[key * nsg + (grp - 2 * ng)];
     const float g = norms[key].y;
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
@@ -273,7 +291,7 @@ struct DScoreLayout {
 };
 DScoreLayout dscore_layout(const tq_quantizer *q, int64_t nq) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
-  const size_t K = (size_t)q->d + q->m;
+  const size_t K = 2 * (size_t)q->d + q->m;
   DScoreLayout L{};
   L.qh = 0;
   L.ql = up((size_t)nq * K * 2);
@@ -297,7 +315,7 @@ tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, 
                       cudaStream_t st) {
   const DScoreLayout L = dscore_layout(q, nq_rows);
   if (!ws || ws_bytes < L.total) return TQ_ERR_WORKSPACE;
-  const int d = q->d, m = q->m, K = d + m, ng = d / 32, nsg = m / 32;
+  const int d = q->d, m = q->m, K = 2 * d + m, ng = d / 32, nsg = m / 32;
   char *base = static_cast<char *>(ws);
   __half *qh = reinterpret_cast<__half *>(base + L.qh), *ql = reinterpret_cast<__half *>(base + L.ql);
   float *qs = reinterpret_cast<float *>(base + L.qs);
@@ -326,7 +344,7 @@ tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, 
     for (int64_t c0 = 0; c0 < nkeys; c0 += kKeyChunk) {
       const int64_t cnt = std::min(kKeyChunk, nkeys - c0);
       const int64_t key0 = g * kpg + key_base + c0;
-      const int64_t threads = cnt * (ng + nsg);
+      const int64_t threads = cnt * (2 * ng + nsg);
       switch (q->w) {
         case 1: k_dscore_keys<1><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(q->kt, cnt, cw + key0 * ng, sw + key0 * nsg, nr + key0, kop); break;
         case 2: k_dscore_keys<2><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(q->kt, cnt, cw + key0 * 2 * ng, sw + key0 * nsg, nr + key0, kop); break;
@@ -341,6 +359,7 @@ tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, 
       prm.M = (int)G;
       prm.N = (int)cnt;
       prm.K = K;
+      prm.d = d;
       prm.nstages = nstages;
       prm.err = q->d_err;
       prm.qscale = qs + g * G;

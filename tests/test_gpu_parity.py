@@ -254,6 +254,33 @@ def test_dense_tensor_core_batches(tq, d, b, rot):
                  d, skip)
 
 
+def test_dense_score_many_queries(tq):
+    """Scoring for d > 128 (tensor-core GEMM over decoded keys): 200 queries (two
+    query tiles, the second ragged) against 3000 keys (ragged key tiles); logits
+    against the oracle, and top-k equal to the sorted logits."""
+    d, b, n, nq = 384, 3, 3000, 200
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((n, d)).astype(np.float32)
+    y = rng.standard_normal((nq, d)).astype(np.float32)
+    t = tables(d, b, "haar")
+    q = tq.tq_codebook(d, b, seed=0, rotation="haar")
+    enc = tq.tq_encode(q, dev(x))
+    rep = check_encode(*host(enc), x, t)
+    s = tq.tq_score(q, dev(y), 1, nq, enc, n)
+    s_ref = o.score(*o.prepare_query(y, t), rep.ref, t)
+    check_scores(s.cpu().numpy(), s_ref, rep.ref["norm"], np.linalg.norm(y, axis=1), d, rep.skip_rows)
+    vals, idx = tq.tq_topk(q, dev(y), enc, 10)
+    sv, si = torch.sort(s, dim=1, descending=True, stable=True)
+    assert torch.equal(vals, sv[:, :10]) and torch.equal(idx, si[:, :10])
+    check_topk(vals.cpu().numpy(), idx.cpu().numpy(), s_ref, rep.ref["norm"], np.linalg.norm(y, axis=1), d, 10)
+    # grouped scoring: 4 groups of 50 queries, each against its own 750 keys
+    sg = tq.tq_score(q, dev(y), 4, 50, enc, 750).cpu().numpy()
+    for g in range(4):
+        ref_g = s_ref[g * 50:(g + 1) * 50, g * 750:(g + 1) * 750]
+        check_scores(sg[g * 50:(g + 1) * 50], ref_g, rep.ref["norm"][g * 750:(g + 1) * 750],
+                     np.linalg.norm(y[g * 50:(g + 1) * 50], axis=1), d, rep.skip_rows[g * 750:(g + 1) * 750])
+
+
 def test_edge_cases(tq):
     t = tables(128, 3)
     q = tq.tq_codebook(128, 3, seed=0)
