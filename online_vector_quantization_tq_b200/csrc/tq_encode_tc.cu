@@ -93,7 +93,7 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }  // namespace
 
 template <int D, int W, int RP, int SRCW, int NXB, bool GATHER>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, D == 32 ? 2 : 1)  // d = 32: two CTAs per SM hide the tile's latency chain
 k_encode_tc(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   using SM = EncSmem<D, RP, SRCW, NXB>;
   constexpr int L = 1 << W;
@@ -416,20 +416,27 @@ tq_status launch_tc(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx
   const int ntiles = (int)((n + kRows - 1) / kRows);
   EncTCParams pp = prm;
   pp.ntiles = ntiles;
-  const int grid = std::min(ntiles, sms);
   if (EncSmem<D, RP, SRCW, 2>::kTotal <= max_smem) {
     auto kern = k_encode_tc<D, W, RP, SRCW, 2, GATHER>;
     const int sm = EncSmem<D, RP, SRCW, 2>::kTotal;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess)
       return TQ_ERR_CUDA;
-    kern<<<grid, kThreads, sm, st>>>(map, pp);
+    // persistent CTAs, as many per SM as fit (each holds 256 TMEM columns);
+    // ask for the largest shared-memory carveout so that two can
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    // (d = 32 is built for two: 128 registers, under half of shared memory
+    // and of TMEM per CTA; the CTAs share nothing, so a pair that cannot be
+    // co-resident would only run one after the other)
+    const int per_sm = D == 32 ? 2 : 1;
+    kern<<<std::min(ntiles, sms * per_sm), kThreads, sm, st>>>(map, pp);
   } else {
     auto kern = k_encode_tc<D, W, RP, SRCW, 1, GATHER>;
     const int sm = EncSmem<D, RP, SRCW, 1>::kTotal;
     if (sm > max_smem) return TQ_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess)
       return TQ_ERR_CUDA;
-    kern<<<grid, kThreads, sm, st>>>(map, pp);
+    kern<<<std::min(ntiles, sms), kThreads, sm, st>>>(map, pp);
   }
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

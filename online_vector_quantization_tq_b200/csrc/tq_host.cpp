@@ -292,6 +292,8 @@ void free_device(tq_quantizer *q) {
   cudaFree(q->d_qjl32);
   cudaFree(q->d_qjl32t);
   q->d_qjl32t = nullptr;
+  cudaFree(q->d_rott);
+  q->d_rott = nullptr;
   q->d_diag_bits = nullptr;
   q->d_rot = nullptr;
   q->d_qjl16 = nullptr;
@@ -445,6 +447,12 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
       for (int j = 0; j < d; ++j) st32[(size_t)j * m + i] = s32[(size_t)i * d + j];
     st = upload(&q->d_qjl32t, st32.data(), st32.size());
   }
+  if (st == TQ_OK && d <= 128) {
+    std::vector<float> rt((size_t)d * d);
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) rt[(size_t)j * d + i] = q->rot[(size_t)i * d + j];
+    st = upload(&q->d_rott, rt.data(), rt.size());
+  }
   if (st == TQ_OK) {
     // Rotation as fp16 pieces for the tensor-core encode.  Hadamard: d^1.5 R
     // is an integer matrix (exact in fp16 when every |entry| <= 2048, else
@@ -559,6 +567,7 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
   kt.qjl16 = q->d_qjl16;
   kt.qjl32 = q->d_qjl32;
   kt.qjl32t = q->d_qjl32t;
+  kt.rott = q->d_rott;
   *out = q;
   return TQ_OK;
 }

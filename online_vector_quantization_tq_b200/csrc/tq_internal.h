@@ -23,6 +23,7 @@ struct KernelTables {
   const uint16_t *qjl16;              // m x d fp16 bit patterns of S
   const float *qjl32;                 // m x d fp32 values of S (same numbers)
   const float *qjl32t;                // d x m: S transposed (coalesced S y~ over rows)
+  const float *rott;                  // d x d: R transposed (d <= 128; coalesced R y over rows)
 };
 
 }  // namespace tq
@@ -42,6 +43,7 @@ struct tq_quantizer {
   uint16_t *d_qjl16 = nullptr;
   float *d_qjl32 = nullptr;
   float *d_qjl32t = nullptr;
+  float *d_rott = nullptr;
   // tensor-core encode: R = tc_rho * (sum of tc_rot_pieces fp16 matrices)
   uint16_t *d_rot16 = nullptr;   // [pieces][d][d] fp16 bits
   int tc_rot_pieces = 0;

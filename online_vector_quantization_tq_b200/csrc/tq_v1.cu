@@ -264,6 +264,41 @@ k_prep_fwht_block(KernelTables kt, RowSource src, int64_t nq, float *ytil, float
   p[row * D + j] = acc0 + acc1;
 }
 
+// Dense rotation, d <= 128: one block per query; y~ = R y walks the
+// transposed R and p = S y~ the transposed S, so every warp load is one
+// contiguous segment.
+__global__ void k_prep_dense_block(KernelTables kt, RowSource src, int64_t nq, float *ytil, float *p) {
+  __shared__ float sv[128];
+  const int d = kt.d, m = kt.m;
+  const int64_t row = blockIdx.x;
+  const int j = threadIdx.x;
+  if (j < d) sv[j] = src.at(row, j);
+  __syncthreads();
+  // four partial sums, eight loads in flight per thread
+  auto dot = [&](const float *mt, int stride, int col) {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    int k = 0;
+    for (; k + 8 <= d; k += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(mt + (size_t)(k + u) * stride + col);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u % 4] = fmaf(v[u], sv[k + u], a[u % 4]);
+    }
+    for (; k < d; ++k) a[0] = fmaf(__ldg(mt + (size_t)k * stride + col), sv[k], a[0]);
+    return (a[0] + a[1]) + (a[2] + a[3]);
+  };
+  float yt = 0.f;
+  if (j < d) yt = dot(kt.rott, d, j);
+  __syncthreads();
+  if (j < d) {
+    sv[j] = yt;
+    ytil[row * d + j] = yt;
+  }
+  __syncthreads();
+  for (int i = j; i < m; i += blockDim.x) p[row * m + i] = dot(kt.qjl32t, m, i);
+}
+
 // ============================================================ score
 // One query row per grid row (blockIdx.y), one key per thread.
 template <int W>
@@ -513,6 +548,12 @@ tq_status v1_prepare_queries(const tq_quantizer *q, const RowSource &src, int64_
       case 64: k_prep_fwht_block<64><<<(unsigned)nq, 64, 0, st>>>(q->kt, src, nq, ytil, p); break;
       case 128: k_prep_fwht_block<128><<<(unsigned)nq, 128, 0, st>>>(q->kt, src, nq, ytil, p); break;
     }
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+  }
+  if (d <= 128 && q->d_rott) {
+    const int threads = std::max(32, (std::max(d, q->m) + 31) / 32 * 32);
+    k_prep_dense_block<<<(unsigned)nq, std::min(threads, 1024), 0, st>>>(q->kt, src, nq, ytil, p);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
   }
