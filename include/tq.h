@@ -152,8 +152,12 @@ tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype,
                     int64_t out_stride, void *stream);
 
 /* Scratch (bytes of device memory) tq_encode needs for n rows; 0 for
- * Hadamard quantizers.  Haar quantizers process rows in batches through
- * this workspace; pass it to tq_encode_ws. */
+ * Hadamard quantizers of d <= 128.  The others (Haar, and Hadamard above
+ * d = 128) process rows in batches through this workspace; pass it to
+ * tq_encode_ws (16-byte aligned; a smaller workspace means smaller batches,
+ * TQ_ERR_WORKSPACE when it cannot hold one).  From d = 256 the batches run
+ * as integer tensor-core GEMMs on 31-bit fixed-point operands (exact
+ * products), up to 32768 rows and about 8*d bytes per row. */
 size_t tq_encode_workspace_bytes(const tq_quantizer *q, int64_t n);
 tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype,
                        int64_t n, int64_t ldx, const int32_t *chan,
@@ -182,7 +186,12 @@ tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq,
  *   receives s = ||x|| * (<y~, c[codes]> + gamma*sqrt(pi/2)/m * <p, 2*bits-1>)
  *   (added to the existing value when accumulate != 0).
  *   workspace: device, at least tq_score_workspace_bytes(q, groups*G) bytes,
- *   16-byte aligned (holds the prepared queries). */
+ *   16-byte aligned (holds the prepared queries; for d > 128 also the
+ *   queries' fp16 pieces and one 32768-key chunk of decoded keys, 2*(2d+m)
+ *   bytes per key, for the tensor-core GEMM that scores them).
+ * Arithmetic: d <= 128 scores with exact integer products of 16-bit
+ * fixed-point limbs; d > 128 with fp16 pieces and fp32 accumulation (error
+ * well inside 1e-3 of max(|s|, ||x|| ||y|| / sqrt(d))). */
 size_t tq_score_workspace_bytes(const tq_quantizer *q, int64_t nq);
 tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups,
                    int64_t G, int64_t ldy, const int32_t *ychan,
