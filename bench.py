@@ -208,6 +208,9 @@ def run_tq(args, rank, world, local):
             for _ in range(max(1, int(0.05 / max(warm_ms * 1e-3, 1e-5)))):
                 step()
             torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
