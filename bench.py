@@ -446,9 +446,9 @@ def run_workload(args):
     print(json.dumps(line), flush=True)
 
 
-# kernels of libtq launched per step: encode (1), query preparation (1), query
-# operand of the integer scorer (1, plus one memset of it), scoring (1)
-LAUNCHES_PER_STEP = 4
+# kernels of libtq launched per step: encode (1), query preparation with the
+# integer scorer's query operand (1), scoring (1)
+LAUNCHES_PER_STEP = 3
 
 
 def _oracle_sample(n_keys):

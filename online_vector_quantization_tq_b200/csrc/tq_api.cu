@@ -173,6 +173,9 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_
   float *ytil = reinterpret_cast<float *>(ws + L.ytil);
   float *p = reinterpret_cast<float *>(ws + L.p);
   RowSource src{y, ldy, ychan, G, q->d, 0};
+  if (tc_score_y_supported(q, G) && aligned(codes, 16) && aligned(signs, 16))
+    return tc_score_y(q, src, groups, G, keys_per_group, codes, signs, norms, out, keys_per_group, accumulate,
+                      reinterpret_cast<int8_t *>(ws + L.qop), reinterpret_cast<float4 *>(ws + L.qsc), s);
   st = v1_prepare_queries(q, src, nq, ytil, p, s);
   if (st != TQ_OK) return st;
   if (tc_score_supported(q, G) && aligned(codes, 16) && aligned(signs, 16))

@@ -56,6 +56,13 @@ tq_status tc2_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ld
                      float *norms, int64_t out_stride, cudaStream_t st);
 
 bool tc_score_supported(const tq_quantizer *q, int64_t G);
+// tq_score from raw queries for Hadamard d = 32, 64, 128: query preparation
+// and the operand fused in one kernel (bit-identical to tc_score after
+// v1_prepare_queries).
+bool tc_score_y_supported(const tq_quantizer *q, int64_t G);
+tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int64_t kpg,
+                     const void *codes, const void *signs, const float *norms, float *out, int64_t ldo,
+                     int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st);
 size_t tc_score_qop_bytes(const tq_quantizer *q, int64_t groups, int64_t G);
 tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
                    int64_t kpg, int64_t key_base, int64_t nkeys, const void *codes, const void *signs,

@@ -114,6 +114,112 @@ k_query_operand(const float *ytil, const float *p, int d, int m, int w, int64_t 
                             (float)(ired[0] + ired[1] + ired[2] + ired[3]), 0.f);
 }
 
+// Query preparation and the query operand in one kernel, for Hadamard
+// quantizers of d = 32, 64, 128: one block of D threads per query.  y~ = R y
+// by three rounds of signs and Walsh-Hadamard butterflies, p = S y~, then the
+// query's five operand rows and its scales.  Every step repeats the
+// arithmetic, in the same order, of the separate preparation
+// (k_prep_fwht_block) and k_query_operand, so the scores are bit-identical
+// whichever way the queries were prepared.
+template <int D>
+__global__ void __launch_bounds__(D)
+k_prep_operand(KernelTables kt, RowSource src, int64_t G, int N, int cexp, int8_t *qop, float4 *qsc) {
+  constexpr int NW = D / 32;
+  __shared__ float v[D];
+  __shared__ float red[2][NW];
+  __shared__ int ired[NW];
+  __shared__ __align__(16) int8_t stg[kColsPerQuery][kScoreKBytes];
+  const int64_t row = blockIdx.x;
+  const int j = threadIdx.x;
+  for (int i = j; i < kColsPerQuery * kScoreKBytes / 16; i += D) reinterpret_cast<uint4 *>(&stg[0][0])[i] = make_uint4(0, 0, 0, 0);
+  float x = src.at(row, j);
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    const uint32_t word = kt.diag_bits[r * (D / 32) + j / 32];
+    x = ((word >> (j % 32)) & 1u) ? -x : x;
+    v[j] = x;
+    __syncthreads();
+#pragma unroll
+    for (int h = 1; h < D; h <<= 1) {
+      const float a = v[j], b = v[j ^ h];
+      x = (j & h) ? b - a : a + b;
+      __syncthreads();
+      v[j] = x;
+      __syncthreads();
+    }
+  }
+  x *= 1.0f / (float(D) * sqrtf(float(D)));
+  v[j] = x;
+  __syncthreads();
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < D; k += 2) {
+    acc0 = fmaf(kt.qjl32t[(size_t)k * D + j], v[k], acc0);
+    acc1 = fmaf(kt.qjl32t[(size_t)(k + 1) * D + j], v[k + 1], acc1);
+  }
+  const float pj = acc0 + acc1;
+  // largest |y~| and |p|: power-of-two scales of the 16-bit fixed point
+  float ay = fabsf(x), ap = fabsf(pj);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ay = fmaxf(ay, __shfl_xor_sync(0xffffffffu, ay, o));
+    ap = fmaxf(ap, __shfl_xor_sync(0xffffffffu, ap, o));
+  }
+  if (j % 32 == 0) {
+    red[0][j / 32] = ay;
+    red[1][j / 32] = ap;
+  }
+  __syncthreads();
+  ay = red[0][0];
+  ap = red[1][0];
+#pragma unroll
+  for (int k = 1; k < NW; ++k) {
+    ay = fmaxf(ay, red[0][k]);
+    ap = fmaxf(ap, red[1][k]);
+  }
+  int ey = 0, ep = 0;
+  frexpf(ay, &ey);
+  frexpf(ap, &ep);
+  const int sy = ay > 0.f ? 14 - ey : 0;
+  const int sp = ap > 0.f ? 14 - ep : 0;
+  {
+    const int vi = __float2int_rn(ldexpf(x, sy));
+    const int hi = (vi + 128) >> 8, lo = vi - 256 * hi;
+    const int k = (j / 32) * 32 + code_byte_pos(kt.w, j % 32);
+    stg[0][k] = (int8_t)hi;
+    stg[1][k] = (int8_t)lo;
+    stg[1][128 + k] = (int8_t)hi;
+    stg[2][128 + k] = (int8_t)lo;
+  }
+  const int pv = __float2int_rn(ldexpf(pj, sp));
+  {
+    const int hi = (pv + 128) >> 8, lo = pv - 256 * hi;
+    const int k = 256 + (j / 32) * 32 + sign_byte_pos(j % 32);
+    stg[3][k] = (int8_t)hi;
+    stg[4][k] = (int8_t)lo;
+  }
+  int psum = pv;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+  if (j % 32 == 0) ired[j / 32] = psum;
+  __syncthreads();
+  // the five rows, 16 bytes at a time, where the 128-byte-swizzled tile keeps them
+  const int64_t g = row / G, ql = row % G;
+  int8_t *img = qop + g * (int64_t)N * kScoreKBytes;
+  const int n0 = kColsPerQuery * (int)ql;
+  for (int t = j; t < kColsPerQuery * (kScoreKBytes / 16); t += D) {
+    const int r = t / (kScoreKBytes / 16), c = t % (kScoreKBytes / 16);
+    *reinterpret_cast<uint4 *>(img + (c / 8) * (N * 128) + sm100::sw128_offset(n0 + r, c % 8)) =
+        *reinterpret_cast<const uint4 *>(&stg[r][16 * c]);
+  }
+  if (j == 0) {
+    int tot = 0;
+#pragma unroll
+    for (int k = 0; k < NW; ++k) tot += ired[k];
+    qsc[row] = make_float4(ldexpf(1.f, -(sy + cexp)), ldexpf(kt.qjl_scale, -sp), (float)tot, 0.f);
+  }
+}
+
 // ------------------------------------------------------------------ key expansion
 namespace {
 
@@ -569,6 +675,12 @@ size_t tc_score_qop_bytes(const tq_quantizer *q, int64_t groups, int64_t G) {
   return (size_t)groups * N * kScoreKBytes;
 }
 
+namespace {
+tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
+                          int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
+                          int64_t ldo, int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st);
+}  // namespace
+
 tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
                    int64_t kpg, int64_t key_base, int64_t nkeys, const void *codes, const void *signs,
                    const float *norms, float *out, int64_t ldo, int accumulate, int8_t *qop, float4 *qsc,
@@ -579,6 +691,35 @@ tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, in
   k_query_operand<<<(unsigned)nq, 128, 0, st>>>(ytil, pq, q->d, q->m, q->w, G, N, q->score_cexp, q->kt.qjl_scale,
                                                 qop, qsc);
   if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+  return tc_score_launch(q, groups, G, kpg, key_base, nkeys, codes, signs, norms, out, ldo, accumulate, qop, qsc,
+                         st);
+}
+
+bool tc_score_y_supported(const tq_quantizer *q, int64_t G) {
+  return tc_score_supported(q, G) && q->rotation == TQ_ROT_HADAMARD && q->d == q->m &&
+         (q->d == 32 || q->d == 64 || q->d == 128) && q->kt.diag_bits;
+}
+
+tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int64_t kpg,
+                     const void *codes, const void *signs, const float *norms, float *out, int64_t ldo,
+                     int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st) {
+  const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
+  const unsigned nq = (unsigned)(groups * G);
+  switch (q->d) {
+    case 32: k_prep_operand<32><<<nq, 32, 0, st>>>(q->kt, src, G, N, q->score_cexp, qop, qsc); break;
+    case 64: k_prep_operand<64><<<nq, 64, 0, st>>>(q->kt, src, G, N, q->score_cexp, qop, qsc); break;
+    case 128: k_prep_operand<128><<<nq, 128, 0, st>>>(q->kt, src, G, N, q->score_cexp, qop, qsc); break;
+    default: return TQ_ERR_UNSUPPORTED;
+  }
+  if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+  return tc_score_launch(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, ldo, accumulate, qop, qsc, st);
+}
+
+namespace {
+tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
+                          int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
+                          int64_t ldo, int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st) {
+  const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   ScoreTCParams prm{};
   prm.d = q->d;
   prm.m = q->m;
@@ -647,5 +788,6 @@ tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, in
 #undef TQ_SC
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
+}  // namespace
 
 }  // namespace tq
