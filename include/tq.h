@@ -67,7 +67,8 @@ typedef enum {
   TQ_ERR_NOMEM = 4,        /* host or device allocation of the quantizer tables failed */
   TQ_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed        */
   TQ_ERR_WORKSPACE = 6,    /* workspace pointer null or smaller than required    */
-  TQ_ERR_TOO_LARGE = 7     /* request needs more than a fixed internal buffer    */
+  TQ_ERR_TOO_LARGE = 7,    /* request needs more than a fixed internal buffer    */
+  TQ_ERR_TIMEOUT = 8       /* a kernel gave up a bounded wait (see tq_sync_check) */
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
@@ -259,6 +260,24 @@ tq_status tq_outlier_channels(const void *x, tq_dtype dtype, int64_t groups,
                               int count, int32_t *out_sel, int32_t *out_rest,
                               void *workspace, size_t workspace_bytes,
                               void *stream);
+
+/* ---------------------------------------------------------------- failures
+ * Every wait inside the tensor-core kernels is bounded (about 2 s).  A kernel
+ * whose wait ran out records a nonzero code in the quantizer's device error
+ * word, stops, frees what it holds and returns; the outputs of that call are
+ * not valid, and the CUDA context stays usable.  (No counterpart in the
+ * TurboQuant pages: this is how the library reports a stalled pipeline.)
+ *
+ * tq_sync_check: synchronizes `stream`, then reads the error word of q.
+ * Returns TQ_OK if no wait ran out since the last check, TQ_ERR_TIMEOUT if
+ * one did (the word is cleared), TQ_ERR_CUDA if the stream itself failed.
+ *
+ * tq_selftest_timeout: launches on `stream` one kernel whose wait can never
+ * be satisfied, so that it runs out (after about 2 s) and records its code:
+ * a test of the failure path that faults and hangs nothing.  Follow it with
+ * tq_sync_check, which then returns TQ_ERR_TIMEOUT. */
+tq_status tq_sync_check(const tq_quantizer *q, void *stream);
+tq_status tq_selftest_timeout(const tq_quantizer *q, void *stream);
 
 #ifdef __cplusplus
 }

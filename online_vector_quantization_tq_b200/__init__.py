@@ -6,4 +6,4 @@ marshalling only).  Build the library with ``build.build()``.
 """
 from .binding import (Encoded, Quantizer, TQError, lib, score_workspace, topk_workspace,  # noqa: F401
                       tq_codebook, tq_codebook_host, tq_encode, tq_outlier_channels,
-                      tq_prepare_queries, tq_score, tq_topk)
+                      tq_prepare_queries, tq_score, tq_selftest_timeout, tq_sync_check, tq_topk)

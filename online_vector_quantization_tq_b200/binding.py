@@ -21,7 +21,8 @@ ROTATIONS = {"auto": 0, "hadamard": 1, "haar": 2}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration",
           3: "misaligned pointer or leading dimension", 4: "out of memory",
           5: "CUDA error", 6: "workspace missing or too small",
-          7: "request exceeds the fixed internal scratch buffer"}
+          7: "request exceeds the fixed internal scratch buffer",
+          8: "a kernel gave up a bounded wait; the outputs of that call are not valid"}
 
 _lib = None
 
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
         "tq_score_noalloc": (i32, [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp, i32, vp]),
         "tq_outlier_workspace_bytes": (sz, [i64, i32]),
         "tq_outlier_channels": (i32, [vp, i32, i64, i64, i32, i64, i32, vp, vp, vp, sz, vp]),
+        "tq_sync_check": (i32, [vp, vp]),
+        "tq_selftest_timeout": (i32, [vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -263,3 +266,14 @@ def tq_outlier_channels(x: torch.Tensor, groups: int, rows_per_group: int, count
         _ptr(x), _dtype(x), groups, rows_per_group, dim, _ld(x), count, _ptr(sel), _ptr(rest),
         _ptr(ws), ws.numel(), _stream(stream)))
     return sel, rest
+
+
+def tq_sync_check(q: "Quantizer", stream=None) -> None:
+    """Synchronize `stream` and raise TQError (status 8) if a kernel of q gave
+    up a bounded wait since the last check (its outputs are not valid)."""
+    _check("tq_sync_check", lib().tq_sync_check(q.handle, _stream(stream)))
+
+
+def tq_selftest_timeout(q: "Quantizer", stream=None) -> None:
+    """Launch a kernel whose wait runs out (about 2 s): tests the failure path."""
+    _check("tq_selftest_timeout", lib().tq_selftest_timeout(q.handle, _stream(stream)))

@@ -334,6 +334,29 @@ tq_status tq_outlier_channels(const void *x, tq_dtype dtype, int64_t groups, int
   return TQ_OK;
 }
 
+
+tq_status tq_sync_check(const tq_quantizer *q, void *stream) {
+  if (!q) return TQ_ERR_INVALID_ARG;
+  if (q->device < 0 || !q->d_err) return TQ_ERR_UNSUPPORTED;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TQ_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, q->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TQ_ERR_CUDA;
+  if (code == 0) return TQ_OK;
+  if (cudaMemset(q->d_err, 0, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_ERR_TIMEOUT;
+}
+
+tq_status tq_selftest_timeout(const tq_quantizer *q, void *stream) {
+  if (!q) return TQ_ERR_INVALID_ARG;
+  if (q->device < 0 || !q->d_err) return TQ_ERR_UNSUPPORTED;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  return launch_wait_selftest(q->d_err, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------- no-allocation scoring

@@ -348,6 +348,7 @@ const char *tq_status_string(tq_status s) {
     case TQ_ERR_CUDA: return "CUDA error";
     case TQ_ERR_WORKSPACE: return "workspace missing or too small";
     case TQ_ERR_TOO_LARGE: return "request exceeds the fixed internal scratch buffer";
+    case TQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait; the outputs of that call are not valid";
   }
   return "unknown status";
 }

@@ -27,6 +27,10 @@ tq_status v1_topk_select(float *score, const int64_t *idx, int64_t rows, int64_t
 tq_status v1_sumsq(const RowSource &src, int64_t groups, int64_t rows_per_group, double *part, int nchunks,
                    double *out, cudaStream_t st);
 
+// One CTA whose mbarrier wait can never complete: the bounded wait runs out
+// and records its code in *err (the failure path, tested without a fault).
+tq_status launch_wait_selftest(int *err, cudaStream_t st);
+
 // cuTensorMapEncodeTiled from the driver (null if unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 

@@ -665,6 +665,24 @@ k_score_tc(const ScoreTCParams p) {
   if (warp == kMmaWarp) sm100::tmem_dealloc(tmem, (uint32_t)tp.ncols);
 }
 
+// ------------------------------------------------------------------ failure self-test
+// An mbarrier expecting one arrival that never comes: the bounded wait gives
+// up after its limit (about 2 s), records code 99 and the kernel returns.
+__global__ void k_wait_selftest(int *err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sm100::mbar_wait(&bar, 0u, err, 99);
+}
+
+tq_status launch_wait_selftest(int *err, cudaStream_t st) {
+  k_wait_selftest<<<1, 32, 0, st>>>(err);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ host side
 bool tc_score_supported(const tq_quantizer *q, int64_t G) {
   return q->d <= 128 && q->d % 32 == 0 && q->m == q->d && G >= 1 && G <= kMaxScoreG;
