@@ -137,17 +137,23 @@ k_prep_operand(KernelTables kt, RowSource src, int64_t G, int N, int cexp, int8_
   for (int r = 0; r < 3; ++r) {
     const uint32_t word = kt.diag_bits[r * (D / 32) + j / 32];
     x = ((word >> (j % 32)) & 1u) ? -x : x;
-    v[j] = x;
-    __syncthreads();
+    // butterflies: partners within a warp by shuffle, across warps through
+    // shared memory (the same a + b and b - a either way)
 #pragma unroll
     for (int h = 1; h < D; h <<= 1) {
-      const float a = v[j], b = v[j ^ h];
-      x = (j & h) ? b - a : a + b;
-      __syncthreads();
-      v[j] = x;
-      __syncthreads();
+      float b;
+      if (h < 32) {
+        b = __shfl_xor_sync(0xffffffffu, x, h);
+      } else {
+        __syncthreads();  // the previous reads of v are done
+        v[j] = x;
+        __syncthreads();
+        b = v[j ^ h];
+      }
+      x = (j & h) ? b - x : x + b;
     }
   }
+  __syncthreads();  // the last butterfly's reads of v are done
   x *= 1.0f / (float(D) * sqrtf(float(D)));
   v[j] = x;
   __syncthreads();
