@@ -293,22 +293,24 @@ __device__ __forceinline__ void expand_codes(const uint32_t *cw, const uint32_t 
 // ------------------------------------------------------------------ scorer
 // Warp-specialised, one persistent CTA per SM walking a contiguous range of
 // 128-key tiles (a group's tiles are contiguous):
-//   warps 0-7    expanders, two groups of four taking alternate tiles; thread
-//                (warp % 4, lane) expands key row 32 (warp % 4) + lane into
-//                its group's key operand in TMEM;
-//   warps 8-15   epilogue, two per TMEM lane quarter, queries split between
+//   warps 0-3    expanders: thread (warp, lane) expands key row 32 warp + lane
+//                into one of the key operands in TMEM (up to four, so the
+//                expanders run ahead of the MMAs; a second group of four
+//                expander warps taking alternate tiles measured no faster);
+//   warps 4-11   epilogue, two per TMEM lane quarter, queries split between
 //                them; scores of a tile from its TMEM accumulator;
-//   warps 16-17  MMA issue, one thread each, alternate tiles (a single issuer
+//   warps 12-13  MMA issue, one thread each, alternate tiles (a single issuer
 //                when only one accumulator fits): an issuing thread spends
 //                tens of cycles per tcgen05 instruction, so two of them keep
 //                the tensor core fed;
-//   warp 18      bulk copies: raw key rows into a ring of kStages buffers, and
+//   warp 14      bulk copies: raw key rows into a ring of kStages buffers, and
 //                each group's query operand into a ring of two.
 // Hand-offs are mbarriers only.  Every wait is bounded and gives up as soon
 // as another role has failed, after which all roles leave their loops,
 // in-flight copies and MMAs are waited for (bounded) and TMEM is freed.
 constexpr int kStages = 4;
-constexpr int kExpWarps = 8, kEpiWarps = 8;
+constexpr int kExpGroups = 1;  // expander groups (four warps each) taking tiles in turn
+constexpr int kExpWarps = 4 * kExpGroups, kEpiWarps = 8;
 constexpr int kMmaWarp = kExpWarps + kEpiWarps;  // and kMmaWarp + 1: the two MMA issuers
 constexpr int kLoadWarp = kMmaWarp + 2;
 constexpr int kScoreThreads = (kLoadWarp + 1) * 32;
@@ -440,7 +442,7 @@ k_score_tc(const ScoreTCParams p) {
       tcl[k] = p.tcl[k];
     }
     TileWalk tw(t0 + e, tpg);
-    for (int it = e; it < n_it; it += 2, tw.advance(2)) {
+    for (int it = e; it < n_it; it += kExpGroups, tw.advance(kExpGroups)) {
       const int64_t g = tw.g, kin = tw.tin * 128 + row;
       const bool valid = kin < p.nkeys;
       uint32_t cw[CW], sw[NG];
