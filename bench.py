@@ -394,7 +394,7 @@ def run_workload(args):
             timed("append", lambda: tq.tq_encode(q, new, out=tail, out_stride=kpg, stream=stream))
             timed("score", lambda: tq.tq_score(q, y, groups, G, cache, kpg, out=out, workspace=ws, stream=stream))
     elif args.workload == "ann":
-        n, d, nq = 1_000_000, 1536, args.queries
+        n, d, nq = args.ann_rows, 1536, args.queries
         x = torch.empty((n, d), device=dev)
         for c in range((n + wl.ANN_CHUNK - 1) // wl.ANN_CHUNK):
             blk = wl.ann_chunk(c, n, d)
@@ -410,7 +410,7 @@ def run_workload(args):
         # the rotation and the QJL projection, and one product per (query, key,
         # coordinate of [y~ | p]): the dense contractions of the step
         flops_ = {"encode": 2.0 * n * d * (d + d), "topk": 2.0 * nq * n * (d + d)}
-        desc = f"ann: 1e6 x 1536 fp32 (std i^-0.5, L2-normalised), Haar, b=4; {nq} queries, top-10"
+        desc = f"ann: {n:,} x 1536 fp32 (std i^-0.5, L2-normalised), Haar, b=4; {nq} queries, top-10"
 
         def step():
             timed("encode", lambda: tq.tq_encode(q, x, out=enc, workspace=wse, stream=stream))
@@ -514,6 +514,8 @@ def main():
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", choices=["kv", "tiny", "kv_mixed", "decode", "ann"], default="kv")
     ap.add_argument("--queries", type=int, default=1024, help="ann workload: number of queries")
+    ap.add_argument("--ann-rows", type=int, default=1_000_000,
+                    help="ann workload: database vectors (1e6 is the workload; fewer for profiling captures)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
