@@ -281,6 +281,40 @@ def test_dense_score_many_queries(tq):
                      np.linalg.norm(y[g * 50:(g + 1) * 50], axis=1), d, rep.skip_rows[g * 750:(g + 1) * 750])
 
 
+@pytest.mark.parametrize("G", [12, 48])
+def test_score_many_heads_per_group(tq, G):
+    """The integer scorer with many queries per group: G = 12 (two accumulators,
+    two key buffers) and G = 48 (one accumulator and one MMA issuer), two groups
+    of 1500 keys (a ragged last tile), and a top-k over 100 queries (batches of
+    48, 48 and 4)."""
+    d, b, kpg, groups = 128, 4, 1500, 2
+    rng = np.random.default_rng(G)
+    x = rng.standard_normal((groups * kpg, d)).astype(np.float32)
+    y = rng.standard_normal((groups * G, d)).astype(np.float32)
+    t = tables(d, b)
+    q = tq.tq_codebook(d, b, seed=0)
+    enc = tq.tq_encode(q, dev(x))
+    rep = check_encode(*host(enc), x, t)
+    s = tq.tq_score(q, dev(y), groups, G, enc, kpg).cpu().numpy()
+    yt = o.prepare_query(y, t)
+    for g in range(groups):
+        rows = slice(g * G, (g + 1) * G)
+        keys = slice(g * kpg, (g + 1) * kpg)
+        ref = {k: v[keys] for k, v in rep.ref.items()}
+        s_ref = o.score(yt[0][rows], yt[1][rows], ref, t)
+        check_scores(s[rows], s_ref, ref["norm"], np.linalg.norm(y[rows], axis=1), d, rep.skip_rows[keys])
+    yq = rng.standard_normal((100, d)).astype(np.float32)
+    n = groups * kpg
+    vals, idx = tq.tq_topk(q, dev(yq), enc, 10)
+    # the same query batches through tq_score use the same kernel: identical logits
+    s_all = torch.cat([tq.tq_score(q, dev(yq[b0:b0 + 48]), 1, len(yq[b0:b0 + 48]), enc, n)
+                       for b0 in range(0, 100, 48)])
+    sv, si = torch.sort(s_all, dim=1, descending=True, stable=True)
+    assert torch.equal(vals, sv[:, :10]) and torch.equal(idx, si[:, :10])
+    s_ref = o.score(*o.prepare_query(yq, t), rep.ref, t)
+    check_topk(vals.cpu().numpy(), idx.cpu().numpy(), s_ref, rep.ref["norm"], np.linalg.norm(yq, axis=1), d, 10)
+
+
 def test_edge_cases(tq):
     t = tables(128, 3)
     q = tq.tq_codebook(128, 3, seed=0)
