@@ -34,6 +34,9 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
   topk .................................. pinned (against an independent
                                           brute-force selection)
   outlier_channels ...................... pinned (planted outliers, ties)
+  boundary_distance ..................... pinned (enumeration over every
+                                          threshold, exact-threshold and
+                                          tail cases, planted off-by-one)
   End-to-end scores on the pages' own workloads: parity unpinned -- the pages
   print no worked numeric example.
 """

@@ -456,3 +456,53 @@ def test_planted_mistakes_are_caught(monkeypatch):
     for stream in (o.STREAM_D1, o.STREAM_D2, o.STREAM_D3):
         v = _fwht_butterfly(v * o.rademacher(11, stream, 32)) / math.sqrt(32)
     assert not np.allclose(x @ r_bad.T, v, atol=1e-12)
+
+
+# ---------------------------------------------------------------- boundary distance
+
+def _brute_boundary_distance(u, thresholds):
+    """min over every threshold t_i of |u - t_i|, by enumeration."""
+    u = np.asarray(u, dtype=np.float64)
+    return np.min(np.abs(u[..., None] - np.asarray(thresholds)[None, :]), axis=-1)
+
+
+@pytest.mark.parametrize("d,b", [(128, 2), (128, 4), (96, 3), (32, 5), (8, 3)])
+def test_boundary_distance_brute_force(d, b):
+    """The exemption rule's distance (what the GPU parity tests forgive) is the
+    distance to the nearest Lloyd-Max threshold (article 1.2.2: a code changes
+    only where u crosses a threshold).  Checked against enumeration on random
+    u, on u exactly at every threshold, just below / above each, below t_0 and
+    above t_last (including |u| = 1)."""
+    t = o.Tables(d, b, seed=3)
+    thr = t.thresholds
+    rng = np.random.default_rng(d * 10 + b)
+    u = rng.uniform(-1.0, 1.0, size=(200, 7)) * rng.choice([1.0, 0.1, 0.01], size=(200, 1))
+    assert np.array_equal(o.boundary_distance(u, t), _brute_boundary_distance(u, thr))
+    eps = 1e-9
+    special_u = np.concatenate([thr, thr - eps, thr + eps, [thr[0] - 0.5, thr[-1] + 0.5, -1.0, 1.0, 0.0]])
+    got = o.boundary_distance(special_u, t)
+    assert np.array_equal(got, _brute_boundary_distance(special_u, thr))
+    assert np.all(got[:thr.size] == 0.0)
+    assert np.allclose(got[thr.size:3 * thr.size], eps, rtol=1e-6) or thr.size == 1
+    # for these u the distance is to the NEAREST threshold: the outer tails
+    # measure to t_0 / t_last, not to a neighbour
+    assert got[3 * thr.size] == pytest.approx(0.5)
+    assert got[3 * thr.size + 1] == pytest.approx(0.5)
+    assert got[3 * thr.size + 2] == pytest.approx(1.0 + thr[0])
+    assert got[3 * thr.size + 3] == pytest.approx(1.0 - thr[-1])
+
+
+def test_boundary_distance_planted_off_by_one(monkeypatch):
+    """An off-by-one in the neighbour index (measuring to t_{j+1} instead of
+    t_j) widens or misplaces the exemption window; the brute-force pin fails."""
+    real = o.boundary_distance
+
+    def off_by_one(u, t):
+        j = np.searchsorted(t.thresholds, u)
+        lo = np.abs(u - t.thresholds[np.clip(j, 0, t.thresholds.size - 1)])
+        hi = np.abs(u - t.thresholds[np.clip(j + 1, 0, t.thresholds.size - 1)])
+        return np.minimum(lo, hi)
+    monkeypatch.setattr(o, "boundary_distance", off_by_one)
+    with pytest.raises(AssertionError):
+        test_boundary_distance_brute_force(128, 4)
+    monkeypatch.setattr(o, "boundary_distance", real)
