@@ -92,6 +92,11 @@ typedef struct {
 /* Human-readable name of a status code (static string, never NULL). */
 const char *tq_status_string(tq_status s);
 
+/* Packed bytes of one encoded vector: codes (w*d/8) + sign bits (m/8) + the
+ * two fp32 norms (8), i.e. what one row occupies across the three output
+ * arrays of tq_encode.  0 for a NULL quantizer.  (tq_info gives the split.) */
+size_t tq_code_bytes(const tq_quantizer *q);
+
 /* ---------------------------------------------------------------- set-up
  * tq_codebook: build a quantizer on the current CUDA device.
  *   d: dimension, a multiple of 32 in [32, 4096]; b: total bits per
@@ -146,7 +151,11 @@ tq_status tq_tables_get(const tq_quantizer *q, float *rotation,
  *      8-byte aligned.
  * Per row: ||x|| (fp32), x_hat = x/||x|| (0 for a zero row), u = R x_hat,
  * code_j = #{thresholds < u_j}, r = u - c[code], gamma = ||r||,
- * sign bit i = [(S r)_i >= 0]. */
+ * sign bit i = [(S r)_i >= 0].
+ * tq_encode takes no workspace and allocates nothing: it serves the
+ * quantizers whose encode needs no scratch (tq_encode_workspace_bytes == 0,
+ * the Hadamard rotation at d <= 128) and returns TQ_ERR_WORKSPACE for the
+ * others, which are encoded with tq_encode_ws and a caller-owned workspace. */
 tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype,
                     int64_t n, int64_t ldx, const int32_t *chan,
                     int64_t chan_rows, void *codes, void *signs, float *norms,
@@ -211,8 +220,13 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups,
  *
  * Scratch comes from one buffer of TQ_NOALLOC_SCRATCH_BYTES compiled into the
  * library as a device variable: every GPU that loads the library holds it
- * until the process exits.  Arguments, layouts and results are exactly those
- * of tq_score.  The call allocates and frees nothing.
+ * until the process exits.  Arguments and layouts are those of tq_score.
+ * Results: for d <= 128 the same kernels run as in tq_score (the integer
+ * tensor-core scorer), so the logits are bit-identical to tq_score's; for
+ * d > 128 the scores come from the CUDA-core scorer (tq_score uses a
+ * tensor-core GEMM there, whose decoded-key chunk does not fit the buffer),
+ * equal to tq_score's within the score tolerance stated at tq_score.  The
+ * call allocates and frees nothing.
  *   - Needed scratch: per query 4*(d + m) + 16 bytes, plus 384 bytes for each
  *     of roundup(5*G, 16) operand rows per group when G <= 48 (each piece
  *     rounded up to 256 bytes).  Larger requests return TQ_ERR_TOO_LARGE

@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
         "tq_codebook_host": (i32, [i32, i32, i32, u64, i32, ctypes.POINTER(vp)]),
         "tq_destroy": (None, [vp]),
         "tq_info": (i32, [vp, ctypes.POINTER(_Info)]),
+        "tq_code_bytes": (sz, [vp]),
         "tq_codebook_get": (i32, [vp, vp, vp, vp]),
         "tq_tables_get": (i32, [vp, vp, vp, vp]),
         "tq_encode": (i32, [vp, vp, i32, i64, i64, vp, i64, vp, vp, vp, i64, vp]),
@@ -242,11 +243,15 @@ def topk_workspace(q: Quantizer, nq: int, n: int, k: int, device="cuda") -> torc
 
 
 def tq_topk(q: Quantizer, y: torch.Tensor, enc: Encoded, k: int, n: int | None = None,
-            workspace: torch.Tensor | None = None, stream=None):
+            workspace: torch.Tensor | None = None, out=None, stream=None):
+    """(scores fp32 [nq, k], key indices int64 [nq, k]); `out` may give both."""
     nq = y.shape[0]
     n = enc.codes.shape[0] if n is None else n
-    vals = torch.empty((nq, k), dtype=torch.float32, device=y.device)
-    idx = torch.empty((nq, k), dtype=torch.int64, device=y.device)
+    if out is None:
+        vals = torch.empty((nq, k), dtype=torch.float32, device=y.device)
+        idx = torch.empty((nq, k), dtype=torch.int64, device=y.device)
+    else:
+        vals, idx = out
     if workspace is None:
         workspace = topk_workspace(q, nq, n, k, y.device)
     _check("tq_topk", lib().tq_topk(

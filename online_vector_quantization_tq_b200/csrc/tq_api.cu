@@ -90,25 +90,20 @@ tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_
                     const int32_t *chan, int64_t chan_rows, void *codes, void *signs, float *norms,
                     int64_t out_stride, void *stream) {
   if (!q) return TQ_ERR_INVALID_ARG;
-  const size_t ws = tq_encode_workspace_bytes(q, n);
-  if (ws == 0)
-    return tq_encode_ws(q, x, dtype, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, nullptr, 0,
-                        stream);
-  bool empty = false;
-  tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows, &empty);
-  if (st != TQ_OK || empty) return st;
-  if (!codes || !signs || !norms || out_stride < 1) return TQ_ERR_INVALID_ARG;
-  DeviceGuard g(q->device);
-  if (!g.ok) return TQ_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  void *buf = nullptr;
-  if (cudaMallocAsync(&buf, ws, s) != cudaSuccess) {
-    cudaGetLastError();
-    return TQ_ERR_NOMEM;
+  // the workspace-free form: quantizers that need scratch are encoded by
+  // tq_encode_ws with caller-owned memory (the library allocates nothing)
+  if (n > 0 && tq_encode_workspace_bytes(q, n) != 0) {
+    bool empty = false;
+    tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows, &empty);
+    return st != TQ_OK ? st : TQ_ERR_WORKSPACE;
   }
-  st = tq_encode_ws(q, x, dtype, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, buf, ws, stream);
-  cudaFreeAsync(buf, s);
-  return st;
+  return tq_encode_ws(q, x, dtype, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, nullptr, 0,
+                      stream);
+}
+
+size_t tq_code_bytes(const tq_quantizer *q) {
+  if (!q) return 0;
+  return (size_t)q->w * q->d / 8 + (size_t)q->m / 8 + 8;
 }
 
 tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy,

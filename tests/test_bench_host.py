@@ -33,3 +33,30 @@ def test_clock_summary_without_samples_says_so():
     cs.error = "no nvidia-smi"
     s = cs.summary()
     assert s["reasons"] == ["unsampled"] and s["sm_mhz"] is None
+
+
+def test_torch_unpackers_match_the_layout_helper():
+    """bench.py's torch unpackers (used by its fp64 quality evaluation) read
+    the packed layout exactly as the tests' numpy helper does."""
+    import numpy as np
+    import torch
+
+    from tests.layout import unpack_codes, unpack_signs
+    b = _bench()
+    rng = np.random.default_rng(0)
+    for d, w in ((128, 1), (128, 2), (96, 3), (64, 3), (32, 4), (1536, 3)):
+        raw = rng.integers(0, 256, size=(7, w * d // 8), dtype=np.uint8)
+        got = b.unpack_codes_t(torch, torch.from_numpy(raw), d, w).numpy()
+        assert np.array_equal(got, unpack_codes(raw, d, w))
+    raw = rng.integers(0, 256, size=(5, 16), dtype=np.uint8)
+    assert np.array_equal(b.unpack_signs_t(torch, torch.from_numpy(raw), 128).numpy(), unpack_signs(raw, 128))
+
+
+def test_traffic_is_null_once_the_source_changes(monkeypatch):
+    b = _bench()
+    digest = b._source_digest("tq_api.cu")
+    monkeypatch.setattr(b, "TRAFFIC", {"k": ("tq_api.cu", digest, 123, "small case"),
+                                       "old": ("tq_api.cu", "0" * 16, 456, "small case")})
+    assert b.traffic_for("k") == (123, "small case")
+    assert b.traffic_for("old") == (None, None)
+    assert b.traffic_for("missing") == (None, None)

@@ -32,6 +32,16 @@ def test_exports_every_declared_symbol(tq):
         assert hasattr(so, name), name
 
 
+@pytest.mark.parametrize("d,b", [(128, 4), (128, 3), (96, 3), (32, 5), (1536, 4)])
+def test_code_bytes(tq, d, b):
+    """Packed bytes per vector = w*d/8 codes + m/8 sign bits + two fp32 norms
+    (72 B for the kv shape d=128, b=4; 776 B for d=1536, b=4)."""
+    q = tq.tq_codebook_host(d, b, seed=0)
+    assert tq.lib().tq_code_bytes(q.handle) == (b - 1) * d // 8 + d // 8 + 8
+    assert tq.lib().tq_code_bytes(q.handle) == q.code_bytes + q.sign_bytes + 8
+    assert tq.lib().tq_code_bytes(None) == 0
+
+
 def test_status_strings(tq):
     L = tq.lib()
     for code in range(7):
