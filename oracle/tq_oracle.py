@@ -33,6 +33,10 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
                                           closed-form variance)
   topk .................................. pinned (against an independent
                                           brute-force selection)
+  TurboQuant-MSE mode (mode="mse") ...... pinned (brute force at d=8, MSE
+                                          against D_b, the shrinkage factor
+                                          1 - d D_b over random rotations,
+                                          and its 2/pi limit at b = 1)
   outlier_channels ...................... pinned (planted outliers, ties)
   boundary_distance ..................... pinned (enumeration over every
                                           threshold, exact-threshold and
@@ -290,15 +294,25 @@ def lloyd_max(d: int, w: int, tol: float = 1e-14, max_iter: int = 100000):
 # ---------------------------------------------------------------------------
 
 class Tables:
-    """Everything a (d, b, m, seed, rotation) quantizer fixes, in float64."""
+    """Everything a (d, b, m, seed, rotation, mode) quantizer fixes, in float64.
+
+    mode "prod" (the default): b - 1 bits to the Lloyd-Max codebook and one
+    QJL bit per coordinate (the inner-product quantizer, TurboQuant article
+    1.2.3).  mode "mse": TurboQuant-MSE, all b bits to the Lloyd-Max codebook
+    and no QJL stage (article 4.1.1 recommends it for most heads at 3 bits,
+    4.2.1 quantizes a vector index with it); there is no S and m = 0."""
 
     def __init__(self, d: int, b: int, m: int | None = None, seed: int = 0,
-                 rotation: str = "auto"):
-        self.d, self.b, self.w = d, b, b - 1
-        self.m = d if m is None else m
+                 rotation: str = "auto", mode: str = "prod"):
+        if mode not in ("prod", "mse"):
+            raise ValueError(f"unknown mode {mode!r}")
+        self.mode = mode
+        self.d, self.b = d, b
+        self.w = b if mode == "mse" else b - 1
+        self.m = 0 if mode == "mse" else (d if m is None else m)
         self.seed = seed
         self.R = rotation_matrix(d, seed, rotation)
-        self.S = qjl_matrix(self.m, d, seed)
+        self.S = qjl_matrix(self.m, d, seed) if mode == "prod" else np.zeros((0, d))
         self.centroids, self.thresholds, self.coord_mse = lloyd_max(d, self.w)
 
 
@@ -326,7 +340,7 @@ def encode(x: np.ndarray, t: Tables) -> dict:
     codes = np.searchsorted(t.thresholds, u, side="left")
     r = u - t.centroids[codes]
     gamma = np.sqrt(np.sum(r * r, axis=1))
-    z = r @ t.S.T
+    z = r @ t.S.T  # (n, 0) in TurboQuant-MSE mode: no sign bits
     bits = z >= 0.0
     return {"codes": codes.astype(np.int64), "bits": bits, "norm": norm,
             "gamma": gamma, "u": u, "z": z}
@@ -355,10 +369,26 @@ def score(ytil: np.ndarray, p: np.ndarray, enc: dict, t: Tables) -> np.ndarray:
     print no constant, so it is derived here).  Returns an nq x n array.
     """
     chat = t.centroids[enc["codes"]]
-    sig = np.where(enc["bits"], 1.0, -1.0)
     mse_term = ytil @ chat.T
+    if t.m == 0:
+        # TurboQuant-MSE (article 4.1.1, 4.2.1): the codebook term alone;
+        # biased, E_R[s] = (1 - d D_b) <y, x> (see mse_inner_product_gain)
+        return enc["norm"][None, :] * mse_term
+    sig = np.where(enc["bits"], 1.0, -1.0)
     qjl_term = (p @ sig.T) * (enc["gamma"][None, :] * math.sqrt(math.pi / 2.0) / t.m)
     return enc["norm"][None, :] * (mse_term + qjl_term)
+
+
+def mse_inner_product_gain(t: Tables) -> float:
+    """E over the rotation of the TurboQuant-MSE estimate divided by <y, x>.
+
+    For a Lloyd-Max codebook every centroid is the mean of its bin, so
+    E[u c(u)] = E[c(u)^2] = E[u^2] - D = 1/d - D per coordinate.  By the
+    rotation's symmetry E_R[R^T c(R x)] is a multiple a x of x, and
+    a = E<u, c(u)> = 1 - d D for a unit x: the estimate shrinks every inner
+    product by the factor 1 - d D_b (the bias the article contrasts with the
+    unbiased inner-product quantizer, 1.2.3)."""
+    return 1.0 - t.d * t.coord_mse
 
 
 def estimator_variance(ytil: np.ndarray, enc: dict, t: Tables) -> np.ndarray:

@@ -506,3 +506,69 @@ def test_boundary_distance_planted_off_by_one(monkeypatch):
     with pytest.raises(AssertionError):
         test_boundary_distance_brute_force(128, 4)
     monkeypatch.setattr(o, "boundary_distance", real)
+
+
+# ---------------------------------------------------------------- TurboQuant-MSE mode
+
+@pytest.mark.parametrize("b", [1, 2, 3])
+def test_mse_mode_brute_force_d8(b):
+    """MSE mode gives all b bits to the codebook: at d = 8 the codes minimise
+    ||u - c[codes]|| over all (2^b)^8 code vectors; no sign bits; the score is
+    ||x|| <y~, c[codes]> (the brute-force nearest codebook point)."""
+    d = 8
+    t = o.Tables(d, b, seed=4, mode="mse")
+    assert t.w == b and t.m == 0 and t.S.shape == (0, d)
+    L = 1 << b
+    grid = np.stack(np.meshgrid(*([np.arange(L)] * d), indexing="ij"), axis=-1).reshape(-1, d)
+    pts = t.centroids[grid]
+    x = np.random.default_rng(b).standard_normal((4, d))
+    y = np.random.default_rng(50 + b).standard_normal((3, d))
+    enc = o.encode(x, t)
+    assert enc["bits"].shape == (4, 0)
+    for i in range(x.shape[0]):
+        best = np.argmin(np.sum((pts - enc["u"][i]) ** 2, axis=1))
+        assert np.array_equal(grid[best], enc["codes"][i])
+    ytil, p = o.prepare_query(y, t)
+    assert p.shape == (3, 0)
+    s = o.score(ytil, p, enc, t)
+    want = (y @ t.R.T) @ (t.centroids[enc["codes"]] * np.linalg.norm(x, axis=1)[:, None]).T
+    assert np.allclose(s, want, rtol=1e-13, atol=1e-13)
+
+
+def test_mse_mode_shrinks_inner_products_by_one_minus_d_D():
+    """Over random Haar rotations the TurboQuant-MSE estimate averages to
+    (1 - d D_b) <y, x> (centroids are bin means); at b = 1 and large d the
+    factor tends to 2/pi.  Checked by simulation for fixed x, y at d = 24."""
+    d, b, trials = 24, 2, 3000
+    t = o.Tables(d, b, seed=0, mode="mse", rotation="haar")
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal(d)
+    y = 0.6 * x + rng.standard_normal(d)  # correlated with x, so <y, x> is far from 0
+    est = np.empty(trials)
+    for s in range(trials):
+        t.R = o.rotation_matrix(d, 1000 + s, "haar")
+        enc = o.encode(x[None, :], t)
+        est[s] = o.score(*o.prepare_query(y[None, :], t), enc, t)[0, 0]
+    want = o.mse_inner_product_gain(t) * float(y @ x)
+    assert abs(est.mean() - want) < 4.0 * est.std() / math.sqrt(trials)
+    # and the factor differs from 1 by far more than that error: the bias is real
+    assert abs(float(y @ x) - want) > 8.0 * est.std() / math.sqrt(trials)
+    # b = 1, large d: 1 - d D_1 -> 2/pi (d D_1 -> 1 - 2/pi for the sign quantizer)
+    _, _, mse = o.lloyd_max(4096, 1)
+    assert abs((1.0 - 4096 * mse) - 2.0 / math.pi) < 2e-4
+
+
+def test_mse_mode_distortion_and_planted_shrinkage_mistake(monkeypatch):
+    """MSE mode encodes with distortion d D_b per unit vector (like the
+    inner-product mode's codebook stage), and a gain formula missing its d
+    factor fails the shrinkage pin."""
+    d, b = 64, 3
+    t = o.Tables(d, b, seed=2, mode="mse")
+    x = _random_unit(20000, d, 3)
+    enc = o.encode(x, t)
+    err = np.sum((x - t.centroids[enc["codes"]] @ t.R) ** 2, axis=1)
+    se = err.std() / math.sqrt(err.size)
+    assert abs(err.mean() - d * t.coord_mse) < 4 * se
+    monkeypatch.setattr(o, "mse_inner_product_gain", lambda tt: 1.0 - tt.coord_mse)
+    with pytest.raises(AssertionError):
+        test_mse_mode_shrinks_inner_products_by_one_minus_d_D()
