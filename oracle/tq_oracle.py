@@ -33,6 +33,9 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
                                           closed-form variance)
   topk .................................. pinned (against an independent
                                           brute-force selection)
+  rerank (two-stage retrieval) .......... pinned (exact top-k by full sort
+                                          when every key is a candidate,
+                                          subsets, ties, planted mistake)
   TurboQuant-MSE mode (mode="mse") ...... pinned (brute force at d=8, MSE
                                           against D_b, the shrinkage factor
                                           1 - d D_b over random rotations,
@@ -442,3 +445,32 @@ def boundary_distance(u: np.ndarray, t: Tables) -> np.ndarray:
     lo = np.abs(u - t.thresholds[np.clip(j - 1, 0, t.thresholds.size - 1)])
     hi = np.abs(u - t.thresholds[np.clip(j, 0, t.thresholds.size - 1)])
     return np.minimum(lo, hi)
+
+
+# ---------------------------------------------------------------------------
+# Two-stage retrieval (TurboQuant article 4.2.2)
+# ---------------------------------------------------------------------------
+
+def rerank(y: np.ndarray, x: np.ndarray, cand: np.ndarray, k: int):
+    """Second stage of two-stage retrieval: the candidates a first stage on
+    the quantized vectors returned are re-scored exactly and the k best kept.
+
+    Article 4.2.2 describes quickly screening a top-K on the quantized
+    vectors, then refining that candidate set; the refinement's measure is
+    not printed.  Reading: the exact inner product <y, x> with the stored
+    raw vectors, in fp64 here; ties to the lower key index; candidate
+    indices < 0 are empty slots.  ``x`` holds the raw database rows indexed
+    by ``cand`` (nq x kc).  Returns (scores, indices), each nq x k, padded
+    with (-inf, -1) when a row has fewer than k valid candidates."""
+    y = np.asarray(y, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    nq = y.shape[0]
+    val = np.full((nq, k), -np.inf)
+    idx = np.full((nq, k), -1, dtype=np.int64)
+    for q in range(nq):
+        c = np.unique(cand[q][cand[q] >= 0])  # ascending: ties go to the lower index
+        s = x[c] @ y[q]
+        order = np.lexsort((c, -s))[:k]
+        val[q, :order.size] = s[order]
+        idx[q, :order.size] = c[order]
+    return val, idx

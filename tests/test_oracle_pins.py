@@ -572,3 +572,39 @@ def test_mse_mode_distortion_and_planted_shrinkage_mistake(monkeypatch):
     monkeypatch.setattr(o, "mse_inner_product_gain", lambda tt: 1.0 - tt.coord_mse)
     with pytest.raises(AssertionError):
         test_mse_mode_shrinks_inner_products_by_one_minus_d_D()
+
+
+# ---------------------------------------------------------------- two-stage retrieval
+
+def test_rerank_equals_exact_topk_when_candidates_cover_it():
+    """With every key a candidate, the second stage is the exact top-k of the
+    raw inner products (brute force by full sort); with a candidate subset
+    it is the exact top-k of that subset; duplicate candidates and empty
+    slots (-1) do not change the result; equal scores go to the lower key."""
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((300, 24))
+    x[200] = x[17]  # an exact tie between keys 17 and 200
+    y = rng.standard_normal((5, 24))
+    y[0] = x[17]
+    every = np.tile(np.arange(300), (5, 1))
+    val, idx = o.rerank(y, x, every, 7)
+    exact = y @ x.T
+    for q in range(5):
+        order = sorted(range(300), key=lambda i: (-exact[q, i], i))[:7]
+        assert idx[q].tolist() == order
+        assert np.allclose(val[q], exact[q, order], rtol=1e-15, atol=0)
+    assert idx[0][:2].tolist() == [17, 200]
+    sub = rng.choice(300, size=(5, 40), replace=True)
+    sub[:, :3] = -1
+    val2, idx2 = o.rerank(y, x, sub, 5)
+    for q in range(5):
+        cs = sorted(set(sub[q][sub[q] >= 0].tolist()), key=lambda i: (-exact[q, i], i))[:5]
+        assert idx2[q].tolist() == cs
+
+
+def test_rerank_planted_mistake(monkeypatch):
+    """A stage that keeps the k smallest instead of the k largest fails."""
+    real = o.rerank
+    monkeypatch.setattr(o, "rerank", lambda y, x, c, k: real(-y, x, c, k))
+    with pytest.raises(AssertionError):
+        test_rerank_equals_exact_topk_when_candidates_cover_it()
