@@ -122,6 +122,20 @@ tq_status tq_codebook(int d, int b, int m, uint64_t seed, tq_rotation rot,
  * device entry points return TQ_ERR_UNSUPPORTED for such a quantizer. */
 tq_status tq_codebook_host(int d, int b, int m, uint64_t seed, tq_rotation rot,
                            tq_quantizer **out);
+/* tq_codebook_mse: a TurboQuant-MSE quantizer (TurboQuant article 4.1.1,
+ * which recommends 3-bit TurboQuant-MSE for most heads, and 4.2.1, which
+ * quantizes a vector index with it): all b bits of a coordinate go to the
+ * Lloyd-Max codebook (w = b, b in [1, 4]) and there is no QJL stage (m = 0,
+ * no sign bits: tq_encode's `signs` and tq_prepare_queries' `p` may be NULL
+ * and are not touched).  The same rotation and codebook fit as tq_codebook.
+ * The score is ||x|| <y~, c[codes]>: biased, every inner product is shrunk
+ * on average by 1 - d D_b (D_b = coord_mse of tq_info), which the
+ * inner-product mode's QJL stage removes.  Supported: encode of bf16 or fp32
+ * keys with the Hadamard rotation at d in {32, 64, 128}; scoring and top-k
+ * at d <= 128.  Other configurations return TQ_ERR_UNSUPPORTED. */
+tq_status tq_codebook_mse(int d, int b, uint64_t seed, tq_rotation rot, tq_quantizer **out);
+tq_status tq_codebook_mse_host(int d, int b, uint64_t seed, tq_rotation rot,
+                               tq_quantizer **out);
 void tq_destroy(tq_quantizer *q);
 tq_status tq_info(const tq_quantizer *q, tq_info_t *info);
 
@@ -249,7 +263,15 @@ tq_status tq_score_noalloc(const tq_quantizer *q, const float *y, int64_t groups
  * 4.2.2, first stage of two-stage retrieval).  y: nq fp32 rows (ldy).
  * out_scores: nq x k fp32, out_idx: nq x k int64 (device), sorted by
  * descending score, equal scores by ascending key index.  1 <= k <= 64 and
- * k <= n.  workspace: at least tq_topk_workspace_bytes(q, nq, n, k) bytes. */
+ * k <= n (the bound of this library's selection kernels; retrieval keeps a
+ * short candidate list).  workspace: at least tq_topk_workspace_bytes(q, nq,
+ * n, k) bytes.  For d > 128 and k <= 16 the selection is fused into the
+ * scoring GEMM: each CTA keeps the 16 best (score, key) pairs per query in
+ * registers and only those candidates reach memory, never the logits; codes
+ * and signs must then be 16-byte aligned (TQ_ERR_ALIGNMENT otherwise).  The
+ * other cases score 65536-key chunks into the workspace and select from
+ * there.  Either way the returned scores are bit-identical to tq_score's
+ * logits of the returned keys. */
 size_t tq_topk_workspace_bytes(const tq_quantizer *q, int64_t nq, int64_t n,
                                int k);
 tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq,
@@ -257,6 +279,26 @@ tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq,
                   const float *norms, int64_t n, int k, float *out_scores,
                   int64_t *out_idx, void *workspace, size_t workspace_bytes,
                   void *stream);
+
+/* ---------------------------------------------------------------- rerank
+ * tq_rerank: the second stage of two-stage retrieval (TurboQuant article
+ * 4.2.2: screen a top-K on the quantized vectors, then refine that candidate
+ * set).  For query i, every candidate key cand[i][c] is re-scored with the
+ * exact inner product <y_i, x_key> against the raw database vectors (fp32
+ * arithmetic), and the k best are written, by descending score, equal
+ * scores by ascending key index.  Typical use: cand = tq_topk's out_idx for
+ * K' > k, x = the vectors that were encoded.
+ *   y: device fp32 [nq][ldy] (ldy >= d); x: device [n][ldx] of `dtype`
+ *   (16-byte aligned, ldx*sizeof(dtype) a multiple of 16, ldx >= d); d a
+ *   multiple of 8.  cand: device int64 [nq][kc], 1 <= kc <= 4096; entries
+ *   outside [0, n) are empty slots and duplicates count once.  out_scores
+ *   fp32 / out_idx int64 [nq][k], 1 <= k <= min(64, kc); a row with fewer
+ *   than k valid candidates is padded with (-inf, -1).  No workspace; the
+ *   call needs no quantizer. */
+tq_status tq_rerank(const float *y, int64_t nq, int64_t ldy, const void *x,
+                    tq_dtype dtype, int64_t n, int64_t ldx, int d,
+                    const int64_t *cand, int kc, int k, float *out_scores,
+                    int64_t *out_idx, void *stream);
 
 /* ---------------------------------------------------------------- outliers
  * tq_outlier_channels: per group of rows, the `count` channels of highest

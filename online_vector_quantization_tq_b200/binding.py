@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
         "tq_status_string": (ctypes.c_char_p, [i32]),
         "tq_codebook": (i32, [i32, i32, i32, u64, i32, ctypes.POINTER(vp)]),
         "tq_codebook_host": (i32, [i32, i32, i32, u64, i32, ctypes.POINTER(vp)]),
+        "tq_codebook_mse": (i32, [i32, i32, u64, i32, ctypes.POINTER(vp)]),
+        "tq_codebook_mse_host": (i32, [i32, i32, u64, i32, ctypes.POINTER(vp)]),
         "tq_destroy": (None, [vp]),
         "tq_info": (i32, [vp, ctypes.POINTER(_Info)]),
         "tq_code_bytes": (sz, [vp]),
@@ -68,6 +70,7 @@ def lib() -> ctypes.CDLL:
         "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
         "tq_topk": (i32, [vp, vp, i64, i64, vp, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
         "tq_score_noalloc": (i32, [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp, i32, vp]),
+        "tq_rerank": (i32, [vp, i64, i64, vp, i32, i64, i64, i32, vp, i32, i32, vp, vp, vp]),
         "tq_outlier_workspace_bytes": (sz, [i64, i32]),
         "tq_outlier_channels": (i32, [vp, i32, i64, i64, i32, i64, i32, vp, vp, vp, sz, vp]),
         "tq_sync_check": (i32, [vp, vp]),
@@ -189,6 +192,19 @@ def tq_codebook_host(d: int, b: int, m: int = 0, seed: int = 0, rotation: str = 
     return Quantizer(h)
 
 
+def tq_codebook_mse(d: int, b: int, seed: int = 0, rotation: str = "auto") -> Quantizer:
+    """TurboQuant-MSE quantizer: all b bits to the codebook, no QJL sign bits."""
+    h = ctypes.c_void_p()
+    _check("tq_codebook_mse", lib().tq_codebook_mse(d, b, seed, ROTATIONS[rotation], ctypes.byref(h)))
+    return Quantizer(h)
+
+
+def tq_codebook_mse_host(d: int, b: int, seed: int = 0, rotation: str = "auto") -> Quantizer:
+    h = ctypes.c_void_p()
+    _check("tq_codebook_mse_host", lib().tq_codebook_mse_host(d, b, seed, ROTATIONS[rotation], ctypes.byref(h)))
+    return Quantizer(h)
+
+
 def tq_encode(q: Quantizer, x: torch.Tensor, out: Encoded | None = None, chan: torch.Tensor | None = None,
               chan_rows: int = 0, out_stride: int = 1, workspace: torch.Tensor | None = None,
               stream=None) -> Encoded:
@@ -257,6 +273,24 @@ def tq_topk(q: Quantizer, y: torch.Tensor, enc: Encoded, k: int, n: int | None =
     _check("tq_topk", lib().tq_topk(
         q.handle, _ptr(y), nq, _ld(y), _ptr(enc.codes), _ptr(enc.signs), _ptr(enc.norms), n, k,
         _ptr(vals), _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return vals, idx
+
+
+def tq_rerank(y: torch.Tensor, x: torch.Tensor, cand: torch.Tensor, k: int, out=None, stream=None):
+    """Second stage of two-stage retrieval: exact <y, x> of every candidate
+    key (cand: int64 [nq, kc], e.g. tq_topk's indices) against the raw rows
+    x, and the k best per query: (scores fp32 [nq, k], keys int64 [nq, k])."""
+    nq, kc = cand.shape
+    if out is None:
+        vals = torch.empty((nq, k), dtype=torch.float32, device=y.device)
+        idx = torch.empty((nq, k), dtype=torch.int64, device=y.device)
+    else:
+        vals, idx = out
+    if cand.dtype != torch.int64 or not cand.is_contiguous():
+        raise TypeError("cand must be a contiguous int64 tensor")
+    _check("tq_rerank", lib().tq_rerank(
+        _ptr(y), nq, _ld(y), _ptr(x), _dtype(x), x.shape[0], _ld(x), x.shape[1], _ptr(cand), kc, k,
+        _ptr(vals), _ptr(idx), _stream(stream)))
     return vals, idx
 
 

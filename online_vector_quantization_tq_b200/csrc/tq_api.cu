@@ -68,12 +68,18 @@ tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype, int
   bool empty = false;
   tq_status st = check_rows(q, x, dtype, n, ldx, chan, chan_rows, &empty);
   if (st != TQ_OK || empty) return st;
-  if (!codes || !signs || !norms || out_stride < 1) return TQ_ERR_INVALID_ARG;
+  if (!codes || (!signs && q->m > 0) || !norms || out_stride < 1) return TQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8)) return TQ_ERR_ALIGNMENT;
   DeviceGuard g(q->device);
   if (!g.ok) return TQ_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   RowSource src{x, ldx, chan, chan_rows, q->d, dtype == TQ_BF16};
+  if (q->m == 0) {  // TurboQuant-MSE: the Hadamard kernels have a variant without the QJL stage
+    if (tc2_encode_supported(q, dtype, chan != nullptr))
+      return tc2_encode(q, x, n, ldx, codes, signs, norms, out_stride, s);
+    if (fwht_fast(q)) return v1_encode_fwht(q, src, n, codes, signs, norms, out_stride, s);
+    return TQ_ERR_UNSUPPORTED;
+  }
   if (tc2_encode_supported(q, dtype, chan != nullptr))
     return tc2_encode(q, x, n, ldx, codes, signs, norms, out_stride, s);
   if (tc_encode_supported(q, dtype, ldx, chan != nullptr))
@@ -111,7 +117,7 @@ tq_status tq_prepare_queries(const tq_quantizer *q, const float *y, int64_t nq, 
   bool empty = false;
   tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, ychan_rows, &empty);
   if (st != TQ_OK || empty) return st;
-  if (!ytil || !p) return TQ_ERR_INVALID_ARG;
+  if (!ytil || (!p && q->m > 0)) return TQ_ERR_INVALID_ARG;
   if (!aligned(ytil, 16) || !aligned(p, 16)) return TQ_ERR_ALIGNMENT;
   DeviceGuard g(q->device);
   if (!g.ok) return TQ_ERR_CUDA;
@@ -155,7 +161,7 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_
   bool empty = false;
   tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, G > 0 ? G : 1, &empty);
   if (st != TQ_OK || empty) return st;
-  if (!codes || !signs || !norms || !out) return TQ_ERR_INVALID_ARG;
+  if (!codes || (!signs && q->m > 0) || !norms || !out) return TQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out, 4)) return TQ_ERR_ALIGNMENT;
   if (nq == 0 || keys_per_group == 0) return TQ_OK;
   if (!workspace || !aligned(workspace, 16) || workspace_bytes < tq_score_workspace_bytes(q, nq))
@@ -195,6 +201,9 @@ struct TopkLayout {
   int64_t chunk, nparts;
 };
 
+// d > 128 with k <= 16: the selection runs inside the scoring GEMM
+inline bool topk_fused_dense(const tq_quantizer *q, int k) { return dense_score_supported(q) && k <= 16; }
+
 TopkLayout topk_layout(const tq_quantizer *q, int64_t nq, int64_t n, int k) {
   TopkLayout L{};
   L.chunk = std::min<int64_t>(n, kTopkChunk);
@@ -204,6 +213,12 @@ TopkLayout topk_layout(const tq_quantizer *q, int64_t nq, int64_t n, int k) {
   off += round_up((size_t)nq * q->d * 4, 256);
   L.p = off;
   off += round_up((size_t)nq * q->m * 4, 256);
+  if (topk_fused_dense(q, k)) {
+    L.dense = off;
+    off += round_up(dense_topk_ws_bytes(q, nq, n), 256);
+    L.total = off;
+    return L;
+  }
   L.qop = off;
   off += round_up((size_t)std::min<int64_t>(nq, 48) * 16 * 384, 256);
   L.qsc = off;
@@ -234,7 +249,7 @@ tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy
   bool empty = false;
   tq_status st = check_rows(q, y, TQ_F32, nq, ldy, nullptr, 0, &empty);
   if (st != TQ_OK || empty) return st;
-  if (n < 0 || !codes || !signs || !norms || !out_scores || !out_idx) return TQ_ERR_INVALID_ARG;
+  if (n < 0 || !codes || (!signs && q->m > 0) || !norms || !out_scores || !out_idx) return TQ_ERR_INVALID_ARG;
   if (k < 1 || k > 64 || k > n) return TQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out_idx, 8) ||
       !aligned(out_scores, 4))
@@ -253,6 +268,11 @@ tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy
   RowSource src{y, ldy, nullptr, 0, q->d, 0};
   st = v1_prepare_queries(q, src, nq, ytil, p, s);
   if (st != TQ_OK) return st;
+  if (topk_fused_dense(q, k)) {
+    if (!aligned(codes, 16) || !aligned(signs, 16)) return TQ_ERR_ALIGNMENT;
+    return dense_topk(q, ytil, p, nq, n, k, codes, signs, norms, out_scores, out_idx, ws + L.dense, L.total - L.dense,
+                      s);
+  }
   const bool tc = tc_score_supported(q, std::min<int64_t>(nq, 48)) && aligned(codes, 16) && aligned(signs, 16);
   const bool dense = !tc && dense_score_supported(q) && aligned(codes, 16) && aligned(signs, 16);
   for (int64_t c0 = 0; c0 < n; c0 += L.chunk) {
@@ -278,6 +298,21 @@ tq_status tq_topk(const tq_quantizer *q, const float *y, int64_t nq, int64_t ldy
   }
   return v1_topk_select(part_s, part_i, nq, L.nparts * k, L.nparts * k, L.nparts * k, 0, k, out_scores, out_idx,
                         k, s);
+}
+
+tq_status tq_rerank(const float *y, int64_t nq, int64_t ldy, const void *x, tq_dtype dtype, int64_t n, int64_t ldx,
+                    int d, const int64_t *cand, int kc, int k, float *out_scores, int64_t *out_idx, void *stream) {
+  if (nq < 0 || n < 0 || d <= 0 || kc < 1 || k < 1 || (dtype != TQ_F32 && dtype != TQ_BF16))
+    return TQ_ERR_INVALID_ARG;
+  if (nq == 0) return TQ_OK;
+  if (!y || !x || !cand || !out_scores || !out_idx || ldy < d || ldx < d) return TQ_ERR_INVALID_ARG;
+  if (k > 64 || k > kc || kc > 4096 || d % 8 != 0 || d > 16384) return TQ_ERR_UNSUPPORTED;
+  const size_t es = dtype == TQ_BF16 ? 2 : 4;
+  if (!aligned(x, 16) || ((size_t)ldx * es) % 16 != 0 || !aligned(cand, 8) || !aligned(out_idx, 8) ||
+      !aligned(out_scores, 4) || !aligned(y, 4))
+    return TQ_ERR_ALIGNMENT;
+  return rerank_launch(y, nq, ldy, x, dtype == TQ_BF16, n, ldx, d, cand, kc, k, out_scores, out_idx,
+                       static_cast<cudaStream_t>(stream));
 }
 
 size_t tq_outlier_workspace_bytes(int64_t groups, int dim) {
@@ -391,7 +426,7 @@ extern "C" tq_status tq_score_noalloc(const tq_quantizer *q, const float *y, int
   bool empty = false;
   tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, G > 0 ? G : 1, &empty);
   if (st != TQ_OK || empty) return st;
-  if (!codes || !signs || !norms || !out) return TQ_ERR_INVALID_ARG;
+  if (!codes || (!signs && q->m > 0) || !norms || !out) return TQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(signs, 4) || !aligned(norms, 8) || !aligned(out, 4)) return TQ_ERR_ALIGNMENT;
   if (keys_per_group == 0) return TQ_OK;
   const bool tc = tc_score_supported(q, G) && aligned(codes, 16) && aligned(signs, 16);

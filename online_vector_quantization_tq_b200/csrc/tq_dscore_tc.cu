@@ -38,6 +38,8 @@ constexpr uint32_t kSABytes = kSBM * kSBK * 2, kSBBytes = kSBN * kSBK * 2;
 constexpr uint32_t kSStage = 2 * kSABytes + kSBBytes;  // query hi, query lo, keys
 constexpr int64_t kKeyChunk = 32768;
 
+constexpr int kTopSlots = 16;  // candidates kept per query row and CTA in top-k mode
+
 struct DScoreParams {
   int M, N, K;  // queries, keys, reduction (2d + m)
   int d;
@@ -48,6 +50,15 @@ struct DScoreParams {
   float *out;           // [M][ldo]
   int64_t ldo;
   int accumulate;
+  // top-k mode (topk != 0): no logits are written.  CTA b owns query tile
+  // b % ntq and key tiles b / ntq, b / ntq + P, ...; each query row keeps
+  // its kTopSlots best (score, key) pairs and writes them to
+  // part_s / part_i [M][part_ld] at column part_base + (b / ntq) * kTopSlots.
+  int topk, P;
+  int64_t key_base;     // index of this chunk's first key
+  float *part_s;
+  int64_t *part_i;
+  int64_t part_ld, part_base;
 };
 
 __global__ void __launch_bounds__(kSThreads, 1)
@@ -63,6 +74,21 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (p.M + kSBM - 1) / kSBM, ntk = (p.N + kSBN - 1) / kSBN;
   const int nitems = ntq * ntk, nk = (p.K + kSBK - 1) / kSBK;
+  // i-th work item of this CTA as (query tile start, key tile start); false when done
+  auto item_at = [&](int i, int &q0, int &k0) {
+    if (p.topk) {
+      const int kt = (int)blockIdx.x / ntq + i * p.P;
+      if ((int)blockIdx.x >= ntq * p.P || kt >= ntk) return false;
+      q0 = ((int)blockIdx.x % ntq) * kSBM;
+      k0 = kt * kSBN;
+      return true;
+    }
+    const int w = (int)blockIdx.x + i * (int)gridDim.x;
+    if (w >= nitems) return false;
+    q0 = (w % ntq) * kSBM;
+    k0 = (w / ntq) * kSBN;
+    return true;
+  };
   const int lo_skip0 = p.d / kSBK, lo_skip1 = 2 * p.d / kSBK;  // K chunks of c_lo
 
   if (threadIdx.x == 0) {
@@ -99,8 +125,8 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
     if (lane == 0) {
       int64_t c = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < nitems && ok; w += gridDim.x) {
-        const int q0 = (w % ntq) * kSBM, k0 = (w / ntq) * kSBN;
+      int q0 = 0, k0 = 0;
+      for (int i = 0; ok && item_at(i, q0, k0); ++i) {
         for (int kc = 0; kc < nk; ++kc, ++c) {
           const int slot = (int)(c % S);
           const int64_t use = c / S;
@@ -122,9 +148,9 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
     if (lane == 0) {
       const uint32_t idesc = sm100::idesc_f16_f32(kSBM, kSBN);
       int64_t c = 0;
-      int item = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++item) {
+      int q0 = 0, k0 = 0;
+      for (int item = 0; ok && item_at(item, q0, k0); ++item) {
         const int ab = item & 1, use = item >> 1;
         if (use > 0 && !wait(&acce[ab], (uint32_t)((use - 1) & 1), 52)) break;
         sm100::tc_fence_after();
@@ -158,15 +184,64 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
     // ------------------------------------------------------------ epilogue
     const int quarter = warp % 4, rin = 32 * quarter + lane;
     const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
-    int item = 0;
-    for (int w = blockIdx.x; w < nitems; w += gridDim.x, ++item) {
-      const int q0 = (w % ntq) * kSBM, k0 = (w / ntq) * kSBN;
+    float *sNorm = reinterpret_cast<float *>(sTmem + 4);  // [2][kSBN] key norms of the item (top-k mode)
+    float ts[kTopSlots];
+    int64_t ti[kTopSlots];
+#pragma unroll
+    for (int j = 0; j < kTopSlots; ++j) {
+      ts[j] = -INFINITY;
+      ti[j] = -1;
+    }
+    int q0 = 0, k0 = 0, qr = -1;
+    for (int item = 0; item_at(item, q0, k0); ++item) {
       const int ab = item & 1, use = item >> 1;
-      const int qr = q0 + rin;
+      qr = q0 + rin;
       const bool valid = qr < p.M;
       const float qs = valid ? p.qscale[qr] : 0.f;
+      if (p.topk) {
+        // the item's key norms, once per CTA, shared by the 128 rows
+        for (int j = threadIdx.x - 64; j < kSBN; j += kSThreads - 64)
+          sNorm[ab * kSBN + j] = k0 + j < p.N ? p.norms[k0 + j].x : 0.f;
+        sm100::named_barrier(1, kSThreads - 64);
+      }
       if (!__all_sync(0xffffffffu, wait(&accf[ab], (uint32_t)(use & 1), 54))) break;
       sm100::tc_fence_after();
+      if (p.topk) {
+        for (int cc = 0; cc < kSBN / 32; ++cc) {
+          const int col0 = k0 + 32 * cc;
+          if (col0 >= p.N) break;  // warp-uniform
+          uint32_t v[32];
+          sm100::tmem_ld32(tmem + tlane + (uint32_t)(ab * kSBN + 32 * cc), v);
+          sm100::tmem_wait_ld();
+          if (!valid) continue;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = col0 + j;
+            // the logit exactly as the all-logits path computes it
+            float sres = __uint_as_float(v[j]) * qs * sNorm[ab * kSBN + 32 * cc + j];
+            if (col < p.N && sres > ts[kTopSlots - 1]) {
+              // keys arrive in ascending index order: an equal score stays
+              // behind the earlier key
+              int64_t id = p.key_base + col;
+#pragma unroll
+              for (int s2 = 0; s2 < kTopSlots; ++s2) {
+                if (sres > ts[s2]) {
+                  const float tv = ts[s2];
+                  const int64_t tix = ti[s2];
+                  ts[s2] = sres;
+                  ti[s2] = id;
+                  sres = tv;
+                  id = tix;
+                }
+              }
+            }
+          }
+        }
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&acce[ab]);
+        continue;
+      }
       float *orow = p.out + (int64_t)qr * p.ldo;
       for (int cc = 0; cc < kSBN / 32; ++cc) {
         const int col0 = k0 + 32 * cc;
@@ -188,6 +263,17 @@ k_dscore_gemm(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ C
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&acce[ab]);
+    }
+    if (p.topk && (int)blockIdx.x < ntq * p.P) {
+      const int row = ((int)blockIdx.x % ntq) * kSBM + rin;
+      if (row < p.M && !*sAbort) {
+        const int64_t o = (int64_t)row * p.part_ld + p.part_base + (int64_t)((int)blockIdx.x / ntq) * kTopSlots;
+#pragma unroll
+        for (int j = 0; j < kTopSlots; ++j) {
+          p.part_s[o + j] = ts[j];
+          p.part_i[o + j] = ti[j];
+        }
+      }
     }
   }
   // ------------------------------------------------------------ teardown
@@ -304,7 +390,7 @@ DScoreLayout dscore_layout(const tq_quantizer *q, int64_t nq) {
 }  // namespace
 
 bool dense_score_supported(const tq_quantizer *q) {
-  return q->d > 128 && q->d % 64 == 0 && q->m % 64 == 0 && q->w >= 1 && q->w <= 4;
+  return q->d > 128 && q->d % 64 == 0 && q->m > 0 && q->m % 64 == 0 && q->w >= 1 && q->w <= 4;
 }
 
 size_t dense_score_ws_bytes(const tq_quantizer *q, int64_t nq) { return dscore_layout(q, nq).total; }
@@ -327,7 +413,7 @@ tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const int extra = 1024 + 8 * 16 + 16;
+  const int extra = 1024 + 8 * 16 + 16 + 2 * kSBN * 4;
   const int nstages = std::min(4, (int)((max_smem - extra) / kSStage));
   if (nstages < 2) return TQ_ERR_UNSUPPORTED;
   const size_t smem = (size_t)nstages * kSStage + extra;
@@ -373,6 +459,93 @@ tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, 
     }
   }
   return TQ_OK;
+}
+
+size_t dense_topk_ws_bytes(const tq_quantizer *q, int64_t nq, int64_t n) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t ntq = (nq + kSBM - 1) / kSBM;
+  const int64_t P = std::max<int64_t>(1, sms / ntq);
+  const int64_t nchunks = (n + kKeyChunk - 1) / kKeyChunk;
+  const size_t slots = (size_t)nchunks * P * kTopSlots;
+  return up(dense_score_ws_bytes(q, nq)) + up((size_t)nq * slots * 4) + up((size_t)nq * slots * 8);
+}
+
+// Top-k over n keys for d > 128 without writing the logits: per 32768-key
+// chunk the keys are decoded and the GEMM keeps, per query row and CTA, the
+// kTopSlots best (score, key) pairs; one selection over those candidates
+// gives the k best (k <= kTopSlots; ties to the lower key index).
+tq_status dense_topk(const tq_quantizer *q, const float *ytil, const float *p, int64_t nq, int64_t n, int k,
+                     const void *codes, const void *signs, const float *norms, float *out_s, int64_t *out_i,
+                     void *ws, size_t ws_bytes, cudaStream_t st) {
+  if (k < 1 || k > kTopSlots) return TQ_ERR_UNSUPPORTED;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  const DScoreLayout L = dscore_layout(q, nq);
+  if (!ws || ws_bytes < dense_topk_ws_bytes(q, nq, n)) return TQ_ERR_WORKSPACE;
+  const int d = q->d, m = q->m, K = 2 * d + m, ng = d / 32, nsg = m / 32;
+  char *base = static_cast<char *>(ws);
+  __half *qh = reinterpret_cast<__half *>(base + L.qh), *ql = reinterpret_cast<__half *>(base + L.ql);
+  float *qs = reinterpret_cast<float *>(base + L.qs);
+  __half *kop = reinterpret_cast<__half *>(base + L.kop);
+  int dev = 0, sms = 0, max_smem = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const int ntq = (int)((nq + kSBM - 1) / kSBM);
+  const int P = std::max(1, sms / ntq);
+  const int64_t nchunks = (n + kKeyChunk - 1) / kKeyChunk;
+  const int64_t slots = nchunks * P * kTopSlots;
+  float *part_s = reinterpret_cast<float *>(base + up(L.total));
+  int64_t *part_i = reinterpret_cast<int64_t *>(base + up(L.total) + up((size_t)nq * slots * 4));
+  k_dscore_queries<<<(unsigned)((nq + 7) / 8), 256, 0, st>>>(ytil, p, d, m, nq, q->kt.qjl_scale, qh, ql, qs);
+  if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+  const int extra = 1024 + 8 * 16 + 16 + 2 * kSBN * 4;
+  const int nstages = std::min(4, (int)((max_smem - extra) / kSStage));
+  if (nstages < 2) return TQ_ERR_UNSUPPORTED;
+  const size_t smem = (size_t)nstages * kSStage + extra;
+  if (cudaFuncSetAttribute(k_dscore_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  CUtensorMap mqh, mql;
+  if (!make_map16(&mqh, qh, K, nq, kSBM) || !make_map16(&mql, ql, K, nq, kSBM)) return TQ_ERR_CUDA;
+  auto cw = static_cast<const uint32_t *>(codes);
+  auto sw = static_cast<const uint32_t *>(signs);
+  auto nr = reinterpret_cast<const float2 *>(norms);
+  for (int64_t ci = 0; ci < nchunks; ++ci) {
+    const int64_t key0 = ci * kKeyChunk;
+    const int64_t cnt = std::min(kKeyChunk, n - key0);
+    const int64_t threads = cnt * (2 * ng + nsg);
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    switch (q->w) {
+      case 1: k_dscore_keys<1><<<blocks, 256, 0, st>>>(q->kt, cnt, cw + key0 * ng, sw + key0 * nsg, nr + key0, kop); break;
+      case 2: k_dscore_keys<2><<<blocks, 256, 0, st>>>(q->kt, cnt, cw + key0 * 2 * ng, sw + key0 * nsg, nr + key0, kop); break;
+      case 3: k_dscore_keys<3><<<blocks, 256, 0, st>>>(q->kt, cnt, cw + key0 * 3 * ng, sw + key0 * nsg, nr + key0, kop); break;
+      case 4: k_dscore_keys<4><<<blocks, 256, 0, st>>>(q->kt, cnt, cw + key0 * 4 * ng, sw + key0 * nsg, nr + key0, kop); break;
+      default: return TQ_ERR_UNSUPPORTED;
+    }
+    if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+    CUtensorMap mk;
+    if (!make_map16(&mk, kop, K, cnt, kSBN)) return TQ_ERR_CUDA;
+    DScoreParams prm{};
+    prm.M = (int)nq;
+    prm.N = (int)cnt;
+    prm.K = K;
+    prm.d = d;
+    prm.nstages = nstages;
+    prm.err = q->d_err;
+    prm.qscale = qs;
+    prm.norms = nr + key0;
+    prm.topk = 1;
+    prm.P = P;
+    prm.key_base = key0;
+    prm.part_s = part_s;
+    prm.part_i = part_i;
+    prm.part_ld = slots;
+    prm.part_base = ci * P * kTopSlots;
+    k_dscore_gemm<<<ntq * P, kSThreads, smem, st>>>(mqh, mql, mk, prm);
+    if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  return v1_topk_select(part_s, part_i, nq, slots, slots, slots, 0, k, out_s, out_i, k, st);
 }
 
 }  // namespace tq

@@ -353,15 +353,24 @@ const char *tq_status_string(tq_status s) {
   return "unknown status";
 }
 
-static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation rot, bool device,
+// mse: TurboQuant-MSE (all b bits to the codebook, no QJL stage, m = 0);
+// otherwise b - 1 codebook bits and an m-row QJL sketch.
+static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation rot, bool device, bool mse,
                                  tq_quantizer **out) {
   using namespace tq;
   if (!out) return TQ_ERR_INVALID_ARG;
   *out = nullptr;
-  if (m == 0) m = d;
-  if (d <= 0 || b < 2 || b > 5 || m <= 0 || (rot != TQ_ROT_AUTO && rot != TQ_ROT_HADAMARD && rot != TQ_ROT_HAAR))
-    return TQ_ERR_INVALID_ARG;
-  if (d % 32 != 0 || d > 4096 || m != d) return TQ_ERR_UNSUPPORTED;
+  if (mse) {
+    if (d <= 0 || b < 1 || b > 4 || (rot != TQ_ROT_AUTO && rot != TQ_ROT_HADAMARD && rot != TQ_ROT_HAAR))
+      return TQ_ERR_INVALID_ARG;
+    m = 0;
+  } else {
+    if (m == 0) m = d;
+    if (d <= 0 || b < 2 || b > 5 || m <= 0 || (rot != TQ_ROT_AUTO && rot != TQ_ROT_HADAMARD && rot != TQ_ROT_HAAR))
+      return TQ_ERR_INVALID_ARG;
+    if (m != d) return TQ_ERR_UNSUPPORTED;
+  }
+  if (d % 32 != 0 || d > 4096) return TQ_ERR_UNSUPPORTED;
   if (rot == TQ_ROT_AUTO) rot = is_pow2(d) ? TQ_ROT_HADAMARD : TQ_ROT_HAAR;
   if (rot == TQ_ROT_HADAMARD && !is_pow2(d)) return TQ_ERR_UNSUPPORTED;
 
@@ -369,7 +378,7 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
   if (!q) return TQ_ERR_NOMEM;
   q->d = d;
   q->b = b;
-  q->w = b - 1;
+  q->w = mse ? b : b - 1;
   q->m = m;
   q->rotation = rot;
   q->seed = seed;
@@ -440,9 +449,9 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
     st = upload(&q->d_diag_bits, bits.data(), bits.size());
   }
   if (st == TQ_OK) st = upload(&q->d_rot, q->rot.data(), q->rot.size());
-  if (st == TQ_OK) st = upload(&q->d_qjl16, q->qjl16.data(), q->qjl16.size());
-  if (st == TQ_OK) st = upload(&q->d_qjl32, s32.data(), s32.size());
-  if (st == TQ_OK) {
+  if (st == TQ_OK && m > 0) st = upload(&q->d_qjl16, q->qjl16.data(), q->qjl16.size());
+  if (st == TQ_OK && m > 0) st = upload(&q->d_qjl32, s32.data(), s32.size());
+  if (st == TQ_OK && m > 0) {
     std::vector<float> st32((size_t)m * d);
     for (int i = 0; i < m; ++i)
       for (int j = 0; j < d; ++j) st32[(size_t)j * m + i] = s32[(size_t)i * d + j];
@@ -521,7 +530,7 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
     for (size_t i = 0; i < sv.size(); ++i) sv[i] = half_bits_to_double(q->qjl16[i]);
     const std::vector<int8_t> rl = limb_split(rv, &q->rot_limb_exp);
     st = upload(&q->d_rot_limbs, rl.data(), rl.size());
-    if (st == TQ_OK) {
+    if (st == TQ_OK && m > 0) {
       const std::vector<int8_t> sl = limb_split(sv, &q->qjl_limb_exp);
       st = upload(&q->d_qjl_limbs, sl.data(), sl.size());
     }
@@ -562,7 +571,7 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
     kt.centroids[i] = i < kt.levels ? (float)q->centroids[i] : 0.0f;
     kt.thresholds[i] = i < kt.levels - 1 ? (float)q->thresholds[i] : INFINITY;
   }
-  kt.qjl_scale = (float)(std::sqrt(M_PI / 2.0) / m);
+  kt.qjl_scale = m > 0 ? (float)(std::sqrt(M_PI / 2.0) / m) : 0.0f;  // no QJL term in TurboQuant-MSE
   kt.diag_bits = q->d_diag_bits;
   kt.rot = q->d_rot;
   kt.qjl16 = q->d_qjl16;
@@ -574,11 +583,19 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
 }
 
 tq_status tq_codebook(int d, int b, int m, uint64_t seed, tq_rotation rot, tq_quantizer **out) {
-  return build_quantizer(d, b, m, seed, rot, true, out);
+  return build_quantizer(d, b, m, seed, rot, true, false, out);
 }
 
 tq_status tq_codebook_host(int d, int b, int m, uint64_t seed, tq_rotation rot, tq_quantizer **out) {
-  return build_quantizer(d, b, m, seed, rot, false, out);
+  return build_quantizer(d, b, m, seed, rot, false, false, out);
+}
+
+tq_status tq_codebook_mse(int d, int b, uint64_t seed, tq_rotation rot, tq_quantizer **out) {
+  return build_quantizer(d, b, 0, seed, rot, true, true, out);
+}
+
+tq_status tq_codebook_mse_host(int d, int b, uint64_t seed, tq_rotation rot, tq_quantizer **out) {
+  return build_quantizer(d, b, 0, seed, rot, false, true, out);
 }
 
 void tq_destroy(tq_quantizer *q) {

@@ -50,6 +50,17 @@ tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, 
                       const float *norms, float *out, int64_t ldo, int accumulate, void *ws, size_t ws_bytes,
                       cudaStream_t st);
 
+// Top-k for d > 128 with the selection fused into the scoring GEMM (no
+// logits in memory); k <= 16.
+size_t dense_topk_ws_bytes(const tq_quantizer *q, int64_t nq, int64_t n);
+tq_status dense_topk(const tq_quantizer *q, const float *ytil, const float *p, int64_t nq, int64_t n, int k,
+                     const void *codes, const void *signs, const float *norms, float *out_s, int64_t *out_i,
+                     void *ws, size_t ws_bytes, cudaStream_t st);
+
+// Exact re-scoring of candidate keys against raw vectors, then top-k.
+tq_status rerank_launch(const float *y, int64_t nq, int64_t ldy, const void *x, bool bf16, int64_t n, int64_t ldx,
+                        int d, const int64_t *cand, int kc, int k, float *out_s, int64_t *out_i, cudaStream_t st);
+
 bool tc_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather);
 tq_status tc_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,
                     int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,

@@ -158,10 +158,12 @@ k_prep_operand(KernelTables kt, RowSource src, int64_t G, int N, int cexp, int8_
   v[j] = x;
   __syncthreads();
   float acc0 = 0.f, acc1 = 0.f;
+  if (kt.m > 0) {  // TurboQuant-MSE quantizers have no QJL projection (p = 0)
 #pragma unroll 8
-  for (int k = 0; k < D; k += 2) {
-    acc0 = fmaf(kt.qjl32t[(size_t)k * D + j], v[k], acc0);
-    acc1 = fmaf(kt.qjl32t[(size_t)(k + 1) * D + j], v[k + 1], acc1);
+    for (int k = 0; k < D; k += 2) {
+      acc0 = fmaf(kt.qjl32t[(size_t)k * D + j], v[k], acc0);
+      acc1 = fmaf(kt.qjl32t[(size_t)(k + 1) * D + j], v[k + 1], acc1);
+    }
   }
   const float pj = acc0 + acc1;
   // largest |y~| and |p|: power-of-two scales of the 16-bit fixed point
@@ -464,11 +466,13 @@ k_score_tc(const ScoreTCParams p) {
             cw[4 * k + 2] = v.z;
             cw[4 * k + 3] = v.w;
           }
-          const uint4 sv = *reinterpret_cast<const uint4 *>(st + SM::kCodeBytes + row * NG * 4);
-          sw[0] = sv.x;
-          sw[1] = sv.y;
-          sw[2] = sv.z;
-          sw[3] = sv.w;
+          if (p.m > 0) {
+            const uint4 sv = *reinterpret_cast<const uint4 *>(st + SM::kCodeBytes + row * NG * 4);
+            sw[0] = sv.x;
+            sw[1] = sv.y;
+            sw[2] = sv.z;
+            sw[3] = sv.w;
+          }
         }
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(&bars[SM::kEmpty + slot]);
@@ -477,8 +481,10 @@ k_score_tc(const ScoreTCParams p) {
           const int64_t key = g * p.kpg + p.key_base + kin;
 #pragma unroll
           for (int k = 0; k < CW; ++k) cw[k] = __ldg(p.codes + key * CW + k);
+          if (p.m > 0) {
 #pragma unroll
-          for (int k = 0; k < NG; ++k) sw[k] = __ldg(p.signs + key * NG + k);
+            for (int k = 0; k < NG; ++k) sw[k] = __ldg(p.signs + key * NG + k);
+          }
         }
       }
       // key operand buffer it % nab was last read by the MMAs of tile it - nab
@@ -494,7 +500,7 @@ k_score_tc(const ScoreTCParams p) {
         for (int k = 0; k < 8; ++k) bt[k] = (sw[gi] >> k) & 0x01010101u;
         sm100::tmem_st8(ta + 8 * gi, ch);
         sm100::tmem_st8(ta + 32 + 8 * gi, cl);
-        sm100::tmem_st8(ta + 64 + 8 * gi, bt);
+        if (p.m > 0) sm100::tmem_st8(ta + 64 + 8 * gi, bt);  // uniform: no sign bytes in TurboQuant-MSE
       }
       sm100::tmem_wait_st();
       sm100::tc_fence_before();
@@ -615,7 +621,8 @@ k_score_tc(const ScoreTCParams p) {
         const uint32_t ta = tmem + (uint32_t)tp.a(ea), td = tmem + (uint32_t)tp.acc(ab);
 #pragma unroll
         for (int ks = 0; ks < kScoreKBytes / 32; ++ks) {
-          if (ks % 4 >= NG) continue;  // coordinates beyond d
+          if (ks % 4 >= NG) continue;       // coordinates beyond d
+          if (ks >= 8 && p.m == 0) continue;  // TurboQuant-MSE: no sign-bit K range
           sm100::mma_i8_ts(td, ta + 8 * ks, bdesc[ks], idesc, ks != 0);
         }
         sm100::mma_commit(&bars[SM::kAEmpty + ea]);
@@ -643,10 +650,10 @@ k_score_tc(const ScoreTCParams p) {
         const int64_t left = p.nkeys - kin0;
         const int rows = left < 128 ? (int)left : 128;
         uint8_t *st = sStage + slot * SM::kStageBytes;
-        const uint32_t cb = rows * CW * 4, sb = rows * NG * 4;
+        const uint32_t cb = rows * CW * 4, sb = p.m > 0 ? rows * NG * 4 : 0;
         sm100::mbar_expect_tx(&bars[SM::kFull + slot], cb + sb);
         sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
-        sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
+        if (sb) sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
       }
     }
   }
@@ -693,7 +700,7 @@ tq_status launch_wait_selftest(int *err, cudaStream_t st) {
 
 // ------------------------------------------------------------------ host side
 bool tc_score_supported(const tq_quantizer *q, int64_t G) {
-  return q->d <= 128 && q->d % 32 == 0 && q->m == q->d && G >= 1 && G <= kMaxScoreG;
+  return q->d <= 128 && q->d % 32 == 0 && (q->m == q->d || q->m == 0) && G >= 1 && G <= kMaxScoreG;
 }
 
 size_t tc_score_qop_bytes(const tq_quantizer *q, int64_t groups, int64_t G) {
@@ -722,7 +729,7 @@ tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, in
 }
 
 bool tc_score_y_supported(const tq_quantizer *q, int64_t G) {
-  return tc_score_supported(q, G) && q->rotation == TQ_ROT_HADAMARD && q->d == q->m &&
+  return tc_score_supported(q, G) && q->rotation == TQ_ROT_HADAMARD &&
          (q->d == 32 || q->d == 64 || q->d == 128) && q->kt.diag_bits;
 }
 
@@ -779,7 +786,7 @@ tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int6
   // bulk copies need 16-byte aligned starts and sizes: with d = 128 a key's
   // code and sign rows are multiples of 16 bytes, so any tile qualifies
   const bool bulk = ng == 4 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
-                    reinterpret_cast<uintptr_t>(signs) % 16 == 0;
+                    (q->m == 0 || reinterpret_cast<uintptr_t>(signs) % 16 == 0);
   if (reinterpret_cast<uintptr_t>(qop) % 16 != 0) return TQ_ERR_ALIGNMENT;
   const size_t smem = 1024 + (bulk ? kStages * stage_bytes : 0) + 2 * (size_t)N * kScoreKBytes + 8 * 48 + 16;
   int dev = 0, sms = 0;

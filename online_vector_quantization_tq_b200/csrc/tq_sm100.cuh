@@ -55,15 +55,27 @@ __device__ __forceinline__ bool mbar_try_wait_for(uint64_t *bar, uint32_t parity
       : "memory");
   return ok != 0;
 }
-constexpr uint32_t kWaitSliceNs = 1000000;  // one sleep of at most 1 ms
-constexpr uint32_t kWaitSlices = 2000;      // about 2 s in all
+constexpr uint32_t kWaitSliceNs = 1000000;      // one sleep of at most 1 ms
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s of wall time in all
+
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 // Bounded wait; on timeout writes `code` to *err (if not yet set) and
-// returns false.
+// returns false.  The limit is wall time measured on the global timer from
+// the first unsuccessful try (the suspend hint of each try is only an upper
+// bound, so counting tries would not bound the time).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code) {
   if (mbar_try_wait(bar, parity)) return true;  // already complete: no sleep
-  for (uint32_t i = 0; i < kWaitSlices; ++i)
+  const uint64_t t0 = global_ns();
+  for (;;) {
     if (mbar_try_wait_for(bar, parity, kWaitSliceNs)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) break;
+  }
   atomicCAS(err, 0, code);
   return false;
 }
@@ -73,9 +85,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
 __device__ __forceinline__ bool mbar_wait_abort(uint64_t *bar, uint32_t parity, volatile int *abort, int *err,
                                                 int code) {
   if (mbar_try_wait(bar, parity)) return true;
-  for (uint32_t i = 0; i < kWaitSlices; ++i) {
+  const uint64_t t0 = global_ns();
+  for (;;) {
     if (mbar_try_wait_for(bar, parity, kWaitSliceNs)) return true;
     if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) break;
   }
   atomicCAS(err, 0, code);
   *abort = 1;
@@ -163,6 +177,19 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// kind::f16 with the A operand (128 rows x 32 bytes = 16 fp16 K elements)
+// read from TMEM: row r in lane r, two consecutive K elements per 32-bit
+// column (the lower K index in the low half).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
@@ -204,6 +231,18 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8])
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
                "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                : "memory");
+}
+// Thread i of the warp writes lane (base lane + i), columns [col, col+32).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -268,6 +307,21 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier over `nthreads` threads that also returns the OR of `pred`
+// over them (a CTA-uniform failure vote for a subset of warps).
+__device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 }  // namespace sm100

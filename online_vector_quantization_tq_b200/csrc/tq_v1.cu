@@ -23,7 +23,7 @@ __global__ void __launch_bounds__(128)
 k_encode_fwht(KernelTables kt, RowSource src, int64_t n, uint32_t *codes, uint32_t *signs,
               float2 *norms, int64_t out_stride) {
   constexpr int L = 1 << W;
-  constexpr int M = D;  // QJL rows
+  const int M = kt.m;  // QJL rows: d, or 0 for TurboQuant-MSE (no sign bits)
   extern __shared__ float4 smem4[];
   float *sS = reinterpret_cast<float *>(smem4);  // M x D fp32
   __shared__ float sC[kMaxLevels];
@@ -258,6 +258,7 @@ k_prep_fwht_block(KernelTables kt, RowSource src, int64_t nq, float *ytil, float
   x *= 1.0f / (float(D) * sqrtf(float(D)));
   v[j] = x;
   ytil[row * D + j] = x;
+  if (kt.m == 0) return;  // TurboQuant-MSE: no QJL projection (uniform over the block)
   __syncthreads();
   // p_j = sum_k S[j][k] y~_k: thread j walks column j of S^T, so every load
   // of the warp is one contiguous segment
@@ -568,6 +569,7 @@ tq_status v1_prepare_queries(const tq_quantizer *q, const RowSource &src, int64_
   EpiStore e1{ytil, d};
   k_gemm_nt<<<dim3(ceil_div_i(nq, 64), ceil_div_i(d, 64)), 256, 0, st>>>(nq, d, d, la, lr, e1);
   TQ_CHECK_LAUNCH();
+  if (q->m == 0) return TQ_OK;  // TurboQuant-MSE: no QJL projection of the query
   LoadMat ly{ytil, d};
   LoadMat ls{q->kt.qjl32, d};
   EpiStore e2{p, q->m};

@@ -21,10 +21,17 @@ def tq():
 def test_bounded_wait_reports_timeout_and_context_survives(tq):
     q = tq.tq_codebook(128, 3, seed=0)
     tq.tq_sync_check(q)  # nothing pending
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
     tq.tq_selftest_timeout(q)
+    b.record()
     with pytest.raises(tq.TQError) as e:
         tq.tq_sync_check(q)
     assert e.value.code == 8
+    # the bound is wall time on the GPU's global timer (2 s), not a count of
+    # suspended tries, so the wait lasts about that long
+    waited = a.elapsed_time(b) / 1e3
+    assert 1.5 <= waited <= 10.0, f"bounded wait lasted {waited:.2f} s"
     tq.tq_sync_check(q)  # the check cleared the word
     # the context still runs the real path: encode + score, then a clean check
     rng = np.random.default_rng(5)

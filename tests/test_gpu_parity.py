@@ -34,6 +34,13 @@ def tables(d, b, rot="auto"):
     return _TABLES[key]
 
 
+def tables_mse(d, b, rot="auto"):
+    key = (d, b, rot, "mse")
+    if key not in _TABLES:
+        _TABLES[key] = o.Tables(d, b, seed=wl.QUANTIZER_SEED, rotation=rot, mode="mse")
+    return _TABLES[key]
+
+
 def host(enc, rows=None):
     sl = slice(None) if rows is None else rows
     return (enc.codes[sl].cpu().numpy(), enc.signs[sl].cpu().numpy(), enc.norms[sl].cpu().numpy())
@@ -299,6 +306,31 @@ def test_dense_score_many_queries(tq):
                      np.linalg.norm(y[g * 50:(g + 1) * 50], axis=1), d, rep.skip_rows[g * 750:(g + 1) * 750])
 
 
+def test_dense_topk_fused_chunks_and_ties(tq):
+    """Top-k for d > 128 with the selection inside the scoring GEMM (no logits
+    in memory): 70000 keys (three 32768-key chunks, the last ragged), 5 and
+    130 queries (one and two query tiles), k = 1, 10, 16 (fused) and 20 (the
+    chunked path); keys 0-499 repeated at 40000-40499 so that equal scores
+    must come out by ascending key index.  Equal to a stable sort of
+    tq_score's logits, bit for bit."""
+    d, b, n = 384, 4, 70000
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((n, d)).astype(np.float32)
+    x[40000:40500] = x[:500]
+    q = tq.tq_codebook(d, b, seed=0, rotation="haar")
+    enc = tq.tq_encode(q, dev(x))
+    for nq in (5, 130):
+        y = dev(rng.standard_normal((nq, d)).astype(np.float32))
+        y[0] = dev(x[7])  # a query whose best keys are the duplicated pair 7 / 40007
+        s = tq.tq_score(q, y, 1, nq, enc, n)
+        sv, si = torch.sort(s, dim=1, descending=True, stable=True)
+        for k in (1, 10, 16, 20):
+            vals, idx = tq.tq_topk(q, y, enc, k)
+            assert torch.equal(vals, sv[:, :k]) and torch.equal(idx, si[:, :k]), (nq, k)
+        vals, idx = tq.tq_topk(q, y, enc, 2)
+        assert idx[0].tolist() == [7, 40007]
+
+
 @pytest.mark.parametrize("G", [12, 48])
 def test_score_many_heads_per_group(tq, G):
     """The integer scorer with many queries per group: G = 12 (two accumulators,
@@ -378,3 +410,133 @@ def test_edge_cases(tq):
                             tq.binding._stream(None))
     assert st == 6
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ TurboQuant-MSE mode
+
+def test_mse_mode_kv_full(tq):
+    """TurboQuant-MSE (all b = 3 bits to the codebook, no QJL sign bits) on
+    the whole kv workload: bf16 keys through the tensor-core encode, codes
+    and norms against the oracle's MSE mode, and every logit of the 32 query
+    heads against the oracle's ||x|| <y~, c[codes]>."""
+    n = 131072
+    xs = _kv_tensor(n)
+    y = wl.kv_queries()
+    t = tables_mse(128, 3)
+    q = tq.tq_codebook_mse(128, 3, seed=0)
+    assert q.sign_bytes == 0 and q.w == 3
+    enc = tq.tq_encode(q, dev(xs.reshape(-1, 128), torch.bfloat16))
+    assert enc.signs.numel() == 0
+    out = tq.tq_score(q, dev(y), 8, 4, enc, n).cpu().numpy()
+    worst = 0.0
+    for h in range(8):
+        rows = slice(h * n, (h + 1) * n)
+        rep = check_encode(*host(enc, rows), xs[h], t)
+        yh = y[4 * h:4 * h + 4]
+        s_ref = o.score(*o.prepare_query(yh, t), rep.ref, t)
+        worst = max(worst, check_scores(out[4 * h:4 * h + 4], s_ref, rep.ref["norm"],
+                                        np.linalg.norm(yh, axis=1), 128, rep.skip_rows))
+    print(f"kv MSE mode: worst score error {worst:.2e}")
+
+
+@pytest.mark.parametrize("d,b", [(128, 2), (64, 4), (32, 1)])
+def test_mse_mode_fp32_and_topk(tq, d, b):
+    """MSE mode for fp32 keys (the CUDA-core Hadamard encode), ragged tiles,
+    a zero key, top-k against the oracle and against the scorer's own
+    logits."""
+    rng = np.random.default_rng(d * 10 + b)
+    x = rng.standard_normal((3001, d)).astype(np.float32)
+    x[9] = 0.0
+    y = rng.standard_normal((7, d)).astype(np.float32)
+    t = tables_mse(d, b)
+    q = tq.tq_codebook_mse(d, b, seed=0)
+    enc = tq.tq_encode(q, dev(x))
+    rep = check_encode(*host(enc), x, t)
+    s = tq.tq_score(q, dev(y), 1, 7, enc, 3001)
+    s_ref = o.score(*o.prepare_query(y, t), rep.ref, t)
+    check_scores(s.cpu().numpy(), s_ref, rep.ref["norm"], np.linalg.norm(y, axis=1), d, rep.skip_rows)
+    vals, idx = tq.tq_topk(q, dev(y), enc, 10)
+    sv, si = torch.sort(s, dim=1, descending=True, stable=True)
+    assert torch.equal(vals, sv[:, :10]) and torch.equal(idx, si[:, :10])
+    check_topk(vals.cpu().numpy(), idx.cpu().numpy(), s_ref, rep.ref["norm"], np.linalg.norm(y, axis=1), d, 10,
+               rep.skip_rows)
+    # an MSE quantizer refuses what it does not support (a Haar rotation)
+    with pytest.raises(tq.TQError) as e:
+        qh = tq.tq_codebook_mse(96, 3, seed=0)
+        tq.tq_encode(qh, dev(rng.standard_normal((10, 96)).astype(np.float32)),
+                     workspace=torch.empty(1 << 20, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == 2
+
+
+# ------------------------------------------------------------------ two-stage retrieval
+
+def _check_rerank(vals, idx, ref_v, ref_i, y, x, k):
+    """Exact inner products in fp32 against fp64: |s - s64| <= (d + 2) 2^-24
+    sum |y_i x_i| (a bound for any summation order); keys equal to the
+    oracle's except where two candidates' exact scores lie within twice that
+    bound of each other."""
+    d = x.shape[1]
+    for q in range(y.shape[0]):
+        bound = (d + 2) * 2.0 ** -24 * (np.abs(x.astype(np.float64)) @ np.abs(y[q].astype(np.float64)))
+        ok = ref_i[q] >= 0
+        assert np.array_equal(idx[q] >= 0, ok)
+        got = idx[q][ok]
+        assert np.all(np.abs(vals[q][ok] - ref_v[q][ok]) <= bound[got])
+        for j in np.nonzero(idx[q] != ref_i[q])[0]:
+            a, b = idx[q][j], ref_i[q][j]
+            assert a >= 0 and b >= 0
+            assert abs(ref_v[q][j] - float(x[a].astype(np.float64) @ y[q])) <= 2 * (bound[a] + bound[b])
+        assert np.all(vals[q][~ok] == -np.inf)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_rerank_against_oracle(tq, dtype):
+    """Second stage on seeded candidate lists (duplicates, empty slots -1 and
+    out-of-range keys included; a row with fewer valid candidates than k),
+    fp32 and bf16 raw vectors, against the oracle's exact re-scoring."""
+    rng = np.random.default_rng(17)
+    n, d, nq, kc, k = 6000, 384, 40, 96, 10
+    x = rng.standard_normal((n, d)).astype(np.float32)
+    if dtype == "bf16":
+        x = wl.to_bf16_values(x)
+    x[123] = x[45]  # an exact tie
+    y = rng.standard_normal((nq, d)).astype(np.float32)
+    cand = rng.integers(0, n, size=(nq, kc))
+    cand[:, 5] = cand[:, 6]        # duplicates
+    cand[0, :2] = (45, 123)
+    y[0] = x[45]
+    cand[1, :] = -1                # a row with three valid candidates
+    cand[1, :3] = (7, 8, 9)
+    cand[2, 10] = n + 5            # out of range: an empty slot
+    xd = dev(x, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    vals, idx = tq.tq_rerank(dev(y), xd, dev(cand, torch.int64), k)
+    vals, idx = vals.cpu().numpy(), idx.cpu().numpy()
+    cand_ref = np.where(cand < n, cand, -1)
+    ref_v, ref_i = o.rerank(y, x, cand_ref, k)
+    _check_rerank(vals, idx, ref_v, ref_i, y, x, k)
+    assert idx[0][:2].tolist() == [45, 123]
+    assert idx[1][3:].tolist() == [-1] * (k - 3)
+
+
+def test_two_stage_retrieval_recall(tq):
+    """Two-stage retrieval on an ANN-shaped sample (d = 1536, the ANN
+    workload's law, 200000 keys, 64 queries): quantized top-100, then exact
+    re-scoring of those 100; recall@10 against exact fp32 inner products is
+    at least the first stage's and reaches 0.97 or more."""
+    n, d, nq = 200000, 1536, 64
+    x = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    for c in range((n + wl.ANN_CHUNK - 1) // wl.ANN_CHUNK):
+        blk = wl.ann_chunk(c, n, d)
+        x[c * wl.ANN_CHUNK:c * wl.ANN_CHUNK + blk.shape[0]] = dev(blk)
+    y = dev(wl.ann_queries(1024, d)[:nq])
+    q = tq.tq_codebook(d, 4, seed=0)
+    enc = tq.tq_encode(q, x)
+    v1, i1 = tq.tq_topk(q, y, enc, 10)
+    vk, ik = tq.tq_topk(q, y, enc, 64)
+    v2, i2 = tq.tq_rerank(y, x, ik, 10)
+    torch.backends.cuda.matmul.allow_tf32 = False
+    truth = torch.topk(y @ x.T, 10, dim=1).indices.cpu().numpy()
+    r1 = np.mean([len(set(a) & set(b)) / 10 for a, b in zip(i1.cpu().numpy(), truth)])
+    r2 = np.mean([len(set(a) & set(b)) / 10 for a, b in zip(i2.cpu().numpy(), truth)])
+    print(f"two-stage: recall@10 first stage {r1:.3f}, after re-scoring the top-64 {r2:.3f}")
+    assert r2 >= r1 and r2 >= 0.97

@@ -110,3 +110,22 @@ def test_layout_is_a_bijection():
     for w in (1, 2, 3, 4):
         pos = sorted(code_bit_position(w, i, b) for i in range(32) for b in range(w))
         assert pos == list(range(32 * w))
+
+
+@pytest.mark.parametrize("d,b", [(128, 3), (64, 1), (128, 4), (96, 2)])
+def test_mse_mode_tables_match_oracle(tq, d, b):
+    """TurboQuant-MSE quantizer: all b bits to the codebook (w = b), no QJL
+    rows (m = 0, no sign bytes), and the same Lloyd-Max fit as the oracle's
+    MSE-mode tables."""
+    q = tq.tq_codebook_mse_host(d, b, seed=0)
+    t = o.Tables(d, b, seed=0, mode="mse")
+    assert (q.w, q.m, q.sign_bytes, q.code_bytes) == (b, 0, 0, b * d // 8)
+    assert tq.lib().tq_code_bytes(q.handle) == b * d // 8 + 8
+    c, thr, mse = q.codebook()
+    scale = np.max(np.abs(t.centroids))
+    assert np.max(np.abs(c - t.centroids)) < 1e-12 * scale
+    assert np.max(np.abs(thr - t.thresholds)) < 1e-12 * scale
+    assert abs(mse - t.coord_mse) < 1e-12 * mse
+    for bad in (0, 5):
+        with pytest.raises(tq.TQError):
+            tq.tq_codebook_mse_host(d, bad, seed=0)
