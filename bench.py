@@ -10,8 +10,10 @@ rank runs its own layer; the path shards by key with no collective).
                   [--workload all|kv|tiny|kv_mixed|decode|ann] [--queries Q]
 
 With the default --workload all, rank 0 of a one-GPU run also times the
-other four workloads (tiny, kv_mixed, decode, ann) and adds one record per
-workload to the headline line under "configs": per-phase CUDA-event times,
+other four workloads (tiny, kv_mixed, decode, ann) and two variants (kv_mse:
+the kv layer with TurboQuant-MSE keys; kv_mixed_2p5: the 2.5-bit outlier
+split) and adds one record per workload to the headline line under
+"configs": per-phase CUDA-event times,
 the roofline of each phase's dominant kernel, quality figures of the encode
 (code decisions and QJL sign bits against an fp64 evaluation, the raw sign
 flip rate of a single-pass fp16 / bf16 projection), the scorer's worst error
@@ -289,6 +291,10 @@ def encode_quality(torch, q, tabs, x, codes_u8, signs_u8, eps=1e-6):
     um = u[cmis]  # distance to the nearest threshold, where the decisions differ
     dist_mis = torch.min((um.unsqueeze(-1) - thr).abs(), dim=-1).values if um.numel() else um
     r = u - c[kc]
+    if m == 0:  # TurboQuant-MSE: codes only
+        return {"keys": int(x.shape[0]), "code_decisions": int(cmis.numel()), "code_mismatch": int(cmis.sum()),
+                "code_mismatch_beyond_eps": int((dist_mis >= eps).sum()),
+                "exempt_fraction": int(cmis.sum()) / max(1, int(cmis.numel()))}
     z = r @ S.T
     ref_bits = z >= 0
     kb = unpack_signs_t(torch, signs_u8, m)
@@ -326,9 +332,12 @@ def score_quality(torch, q, tabs, y, codes_u8, signs_u8, norms, logits):
     ytil = y.double() @ R.T
     p = ytil @ S.T
     chat = c[unpack_codes_t(torch, codes_u8, q.d, q.w)]
-    sig = unpack_signs_t(torch, signs_u8, q.m).double() * 2.0 - 1.0
     xn, gam = norms[:, 0].double(), norms[:, 1].double()
-    s64 = xn[None, :] * (ytil @ chat.T + (p @ sig.T) * (gam[None, :] * math.sqrt(math.pi / 2.0) / q.m))
+    if q.m == 0:  # TurboQuant-MSE: the codebook term alone
+        s64 = xn[None, :] * (ytil @ chat.T)
+    else:
+        sig = unpack_signs_t(torch, signs_u8, q.m).double() * 2.0 - 1.0
+        s64 = xn[None, :] * (ytil @ chat.T + (p @ sig.T) * (gam[None, :] * math.sqrt(math.pi / 2.0) / q.m))
     err = (logits.double() - s64).abs()
     floor = torch.linalg.norm(y.double(), dim=1)[:, None] * xn[None, :] / math.sqrt(q.d)
     plain = err / s64.abs().clamp_min(1e-300)
@@ -405,8 +414,20 @@ def oracle_rate_for(name):
             dt = time.perf_counter() - t0
             return {"value": x.shape[0] / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
                     "sample": f"the whole workload: 4096 keys encoded + 16 queries top-10, {dt:.2f} s"}
-        if name == "kv_mixed":
-            ta, tb = o.Tables(32, 5, seed=0), o.Tables(96, 3, seed=0)
+        if name == "kv_mse":
+            t = o.Tables(128, 3, seed=0, mode="mse")
+            n = 32768
+            x = wl.kv_head_keys(0, 131072)[:n]
+            y = wl.kv_queries()[:4]
+            t0 = time.perf_counter()
+            enc = o.encode(x, t)
+            o.score(*o.prepare_query(y, t), enc, t)
+            dt = time.perf_counter() - t0
+            return {"value": n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
+                    "sample": f"{n} keys of KV head 0 encoded (MSE mode) + scored by 4 query heads, {dt:.2f} s"}
+        if name in ("kv_mixed", "kv_mixed_2p5"):
+            (da, ba), (db, bb) = ((32, 5), (96, 3)) if name == "kv_mixed" else ((32, 4), (96, 2))
+            ta, tb = o.Tables(da, ba, seed=0), o.Tables(db, bb, seed=0)
             n = 16384
             x = wl.kv_head_keys(0, 131072)[:n]
             y = wl.kv_queries()[:4]
@@ -632,13 +653,15 @@ def run_config(name, args, torch, tq, dev, stream, peak):
         logits = tq.tq_score(q, y, 1, 16, enc, n)
         rec["quality"] = {"encode": encode_quality(torch, q, tabs, x, enc.codes, enc.signs),
                           "score": score_quality(torch, q, tabs, y, enc.codes, enc.signs, enc.norms, logits)}
-    elif name == "kv_mixed":
+    elif name in ("kv_mixed", "kv_mixed_2p5"):
         kpg, groups, G = 131072, 8, 4
+        (da, ba), (db, bb) = ((32, 5), (96, 3)) if name == "kv_mixed" else ((32, 4), (96, 2))
+        bits = (da * (ba) + db * bb) / 128.0
         xs, y_np = kv_keys_host()
         x = torch.from_numpy(xs).to(dev).to(torch.bfloat16)
         y = torch.from_numpy(y_np).to(dev)
         sel, rest = tq.tq_outlier_channels(x, groups, kpg, 32)
-        qa, qb = tq.tq_codebook(32, 5, seed=0), tq.tq_codebook(96, 3, seed=0)
+        qa, qb = tq.tq_codebook(da, ba, seed=0), tq.tq_codebook(db, bb, seed=0)
         n = x.shape[0]
         encs = [(qa.empty_encoded(n, dev), qb.empty_encoded(n, dev)) for _ in range(2)]
         out = torch.empty((groups * G, kpg), device=dev)
@@ -646,38 +669,81 @@ def run_config(name, args, torch, tq, dev, stream, peak):
         wse = torch.empty(max(16, tq.lib().tq_encode_workspace_bytes(qb.handle, n)), dtype=torch.uint8,
                           device=dev)
         it = [0]
+        pa, pb = f"encode_d{da}_b{ba}", f"encode_d{db}_b{bb}"
 
         def step():
             i = it[0]
             it[0] += 1
             (ea, eb), (ra, rb) = encs[i % 2], encs[(i + 1) % 2]
-            ph("encode_d32_b5", lambda: tq.tq_encode(qa, x, out=ea, chan=sel, chan_rows=kpg, stream=stream))
-            ph("encode_d96_b3", lambda: tq.tq_encode(qb, x, out=eb, chan=rest, chan_rows=kpg, workspace=wse,
-                                                     stream=stream))
+            ph(pa, lambda: tq.tq_encode(qa, x, out=ea, chan=sel, chan_rows=kpg, stream=stream))
+            ph(pb, lambda: tq.tq_encode(qb, x, out=eb, chan=rest, chan_rows=kpg, workspace=wse, stream=stream))
             ph("score", lambda: (tq.tq_score(qa, y, groups, G, ra, kpg, out=out, ychan=sel, workspace=wsa,
                                              stream=stream),
                                  tq.tq_score(qb, y, groups, G, rb, kpg, out=out, accumulate=True, ychan=rest,
                                              workspace=wsb, stream=stream)))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
         pm = ph.mean_ms()
-        enc_ms = pm["encode_d32_b5"] + pm["encode_d96_b3"]
-        rec = {"workload": "kv_mixed: kv tensors, per head the 32 highest-RMS channels at b=5 (d=32, Hadamard) + "
-                           "96 at b=3 (d=96, Haar), scores summed",
+        enc_ms = pm[pa] + pm[pb]
+        key_b = qa.code_bytes + qa.sign_bytes + 8 + qb.code_bytes + qb.sign_bytes + 8
+        rec = {"workload": f"{name}: kv tensors, per head the 32 highest-RMS channels at b={ba} (d=32, Hadamard) "
+                           f"+ 96 at b={bb} (d=96, Haar), scores summed ({bits:g} bits per channel)",
                "value": n / (ms * 1e-3), "unit": "keys/s", "ms_per_step": ms, "phases_ms": pm,
                "encode_vectors_per_s": n / (enc_ms * 1e-3), "score_keys_per_s": n / (pm["score"] * 1e-3),
+               "bytes_per_key": key_b,
                "l2": "two code buffers; each step scores the codes encoded one step earlier",
-               "roofline": {"encode": roofline_hbm(n * 328, enc_ms, peak, "k_encode_tc",
-                                                   "328 B/key (256 in; 16+4+8 and 24+12+8 out), both parts"),
-                            "score": roofline_hbm(n * 88, pm["score"], peak, "k_score_tc",
-                                                  "88 B/key (72 in, 16 logits out), both parts")}}
+               "roofline": {"encode": roofline_hbm(n * (256 + key_b), enc_ms, peak, "k_encode_tc",
+                                                   f"{256 + key_b} B/key (256 in, {key_b} out), both parts"),
+                            "score": roofline_hbm(n * (key_b + 16), pm["score"], peak, "k_score_tc",
+                                                  f"{key_b + 16} B/key ({key_b} in, 16 logits out), both parts")}}
         ea, eb = encs[0]
         rows = torch.arange(0, kpg, 4, device=dev)  # 32768 keys of head 0
         xa = x[rows][:, sel[0].long()]
         xb = x[rows][:, rest[0].long()]
         tabs_a, tabs_b = quantizer_tables_t(torch, qa, dev), quantizer_tables_t(torch, qb, dev)
-        rec["quality"] = {"encode_d32_b5": encode_quality(torch, qa, tabs_a, xa, ea.codes[rows], ea.signs[rows]),
-                          "encode_d96_b3": encode_quality(torch, qb, tabs_b, xb, eb.codes[rows], eb.signs[rows]),
+        rec["quality"] = {pa: encode_quality(torch, qa, tabs_a, xa, ea.codes[rows], ea.signs[rows]),
+                          pb: encode_quality(torch, qb, tabs_b, xb, eb.codes[rows], eb.signs[rows]),
                           "sample": "every 4th key of KV head 0"}
+    elif name == "kv_mse":
+        groups, G, kpg, b = 8, 4, 131072, 3
+        xs, y_np = kv_keys_host()
+        x = torch.from_numpy(xs).to(dev).to(torch.bfloat16)
+        y = torch.from_numpy(y_np).to(dev)
+        q = tq.tq_codebook_mse(128, b, seed=0)
+        n = x.shape[0]
+        encs = [q.empty_encoded(n, dev) for _ in range(2)]
+        logits = torch.empty((groups * G, kpg), dtype=torch.float32, device=dev)
+        ws = tq.score_workspace(q, groups * G, dev)
+        it = [0]
+
+        def step():
+            i = it[0]
+            it[0] += 1
+            ph("encode", lambda: tq.tq_encode(q, x, out=encs[i % 2], stream=stream))
+            ph("score", lambda: tq.tq_score(q, y, groups, G, encs[(i + 1) % 2], kpg, out=logits, workspace=ws,
+                                            stream=stream))
+        ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        pm = ph.mean_ms()
+        kb = q.code_bytes + 8
+        rec = {"workload": "kv_mse: the kv workload with TurboQuant-MSE keys (b = 3 bits all to the codebook, no QJL "
+                           "stage), 32 query heads, all fp32 logits",
+               "value": n / (ms * 1e-3), "unit": "keys/s", "ms_per_step": ms, "phases_ms": pm,
+               "encode_vectors_per_s": n / (pm["encode"] * 1e-3), "score_keys_per_s": n / (pm["score"] * 1e-3),
+               "bytes_per_key": kb,
+               "l2": "two code buffers; each step scores the codes encoded one step earlier",
+               "roofline": {"encode": roofline_hbm(n * (256 + kb), pm["encode"], peak, "k_encode_tc2",
+                                                   f"{256 + kb} B/key (256 in, 48 codes + 8 norms out)"),
+                            "score": roofline_hbm(n * (kb + 16), pm["score"], peak, "k_score_tc",
+                                                  f"{kb + 16} B/key ({kb} in, 16 logits out)")}}
+        tabs = quantizer_tables_t(torch, q, dev)
+        rows = torch.arange(0, n, 16, device=dev)
+        e = encs[0]
+        sc = tq.tq_score(q, y[:4], 1, 4, tq.binding.Encoded(e.codes[:kpg:4], e.signs[:kpg:4], e.norms[:kpg:4]),
+                         kpg // 4)
+        rec["quality"] = {"encode": encode_quality(torch, q, tabs, x[rows], e.codes[rows], e.signs[rows]),
+                          "score": score_quality(torch, q, tabs, y[:4], e.codes[:kpg:4], e.signs[:kpg:4],
+                                                 e.norms[:kpg:4], sc),
+                          "inner_product_gain_1_minus_dD": 1.0 - 128 * q.coord_mse,
+                          "sample": "encode: every 16th key; score: query heads 0-3 x every 4th key of KV head 0"}
     elif name == "decode":
         groups, kpg, G = 256, 32768, 4
         q = tq.tq_codebook(128, 3, seed=0)
@@ -762,6 +828,23 @@ def run_config(name, args, torch, tq, dev, stream, peak):
         truth = torch.cat(truth)
         hits = sum(len(set(a) & set(b)) for a, b in zip(idx.cpu().tolist(), truth.cpu().tolist()))
         rec["recall_at_10_vs_exact_fp32"] = hits / (10.0 * nq)
+        # two-stage retrieval: the quantized top-16, then exact re-scoring of those 16
+        ws16 = tq.topk_workspace(q, nq, n, 16, dev)
+        v16 = torch.empty((nq, 16), device=dev)
+        i16 = torch.empty((nq, 16), dtype=torch.int64, device=dev)
+        v2 = torch.empty((nq, 10), device=dev)
+        i2 = torch.empty((nq, 10), dtype=torch.int64, device=dev)
+        ph2 = Phases(torch, stream)
+
+        def two_stage():
+            ph2("topk16", lambda: tq.tq_topk(q, y, enc, 16, workspace=ws16, out=(v16, i16), stream=stream))
+            ph2("rerank", lambda: tq.tq_rerank(y, x, i16, 10, out=(v2, i2), stream=stream))
+        timed_steps(torch, dev, stream, two_stage, min(steps, 5), 2, ph2)
+        hits2 = sum(len(set(a) & set(b)) for a, b in zip(i2.cpu().tolist(), truth.cpu().tolist()))
+        rec["two_stage"] = {"first_stage_k": 16, "phases_ms": ph2.mean_ms(),
+                            "recall_at_10_vs_exact_fp32": hits2 / (10.0 * nq),
+                            "note": "exact fp32 inner products of the 16 quantized candidates against the raw "
+                                    "vectors (TurboQuant article 4.2.2, second stage)"}
         tabs = quantizer_tables_t(torch, q, dev)
         rows = torch.arange(0, n, max(1, n // 16384), device=dev)[:16384]
         logits = tq.tq_score(q, y[:16], 1, 16, tq.binding.Encoded(enc.codes[rows], enc.signs[rows],
@@ -815,7 +898,7 @@ def run_tq(args, rank, world, local):
                                   "phases_ms": {"encode": line["encode_ms"], "score": line["score_ms"]},
                                   "roofline": {"encode": line["roofline"], "score": line["score_roofline"]},
                                   "quality": quality, "cpu_baseline": line["cpu_baseline"]}}
-                for name in ("tiny", "kv_mixed", "decode", "ann"):
+                for name in ("tiny", "kv_mixed", "decode", "ann", "kv_mse", "kv_mixed_2p5"):
                     configs[name] = run_config(name, args, torch, tq, dev, stream, peak)
                     torch.cuda.empty_cache()
                 line["configs"] = configs
@@ -852,7 +935,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--workload", choices=["all", "kv", "tiny", "kv_mixed", "decode", "ann"], default="all")
+    ap.add_argument("--workload", choices=["all", "kv", "tiny", "kv_mixed", "decode", "ann", "kv_mse",
+                                           "kv_mixed_2p5"], default="all")
     ap.add_argument("--queries", type=int, default=1024, help="ann workload: number of queries")
     ap.add_argument("--ann-rows", type=int, default=1_000_000,
                     help="ann workload: database vectors (1e6 is the workload; fewer for profiling captures)")

@@ -84,6 +84,7 @@ tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype, int
     return tc2_encode(q, x, n, ldx, codes, signs, norms, out_stride, s);
   if (tc_encode_supported(q, dtype, ldx, chan != nullptr))
     return tc_encode(q, x, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, s);
+  if (fwht_tc_encode_supported(q)) return fwht_tc_encode(q, src, n, codes, signs, norms, out_stride, s);
   if (fwht_fast(q)) return v1_encode_fwht(q, src, n, codes, signs, norms, out_stride, s);
   if (!workspace || !aligned(workspace, 16)) return TQ_ERR_WORKSPACE;
   if (dense_tc_supported(q))

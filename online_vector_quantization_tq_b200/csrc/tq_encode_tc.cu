@@ -72,18 +72,6 @@ constexpr int split_point() {
   return 32 * ((D / 32 + 1) / 2);
 }
 
-// Copy a row-major fp16 [rows][D] matrix from global memory into a 64-byte
-// swizzled K-major operand (D/32 blocks of rows x 64 B).
-template <int D>
-__device__ void stage_kmajor(uint8_t *dst, const uint16_t *src, int rows) {
-  const int chunks = rows * (D / 8);
-  for (int i = threadIdx.x; i < chunks; i += blockDim.x) {
-    const int r = i / (D / 8), c8 = i % (D / 8);  // 8-element chunk index along K
-    const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * D + c8 * 8);
-    const int blk = c8 / 4, ch = c8 % 4;
-    *reinterpret_cast<uint4 *>(dst + (size_t)blk * rows * 64 + sm100::sw64_offset(r, ch)) = v;
-  }
-}
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -131,8 +119,8 @@ k_encode_tc(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   }
   if (tid < kMaxLevels) sCen[tid] = p.cen_s[tid];
 #pragma unroll
-  for (int pc = 0; pc < RP; ++pc) stage_kmajor<D>(sBr + pc * (D * D * 2), p.rot16 + (size_t)pc * D * D, D);
-  stage_kmajor<D>(sBs, p.s16, D);
+  for (int pc = 0; pc < RP; ++pc) sm100::stage_kmajor<D>(sBr + pc * (D * D * 2), p.rot16 + (size_t)pc * D * D, D);
+  sm100::stage_kmajor<D>(sBs, p.s16, D);
   sm100::fence_proxy_async();
   sm100::tc_fence_before();
   __syncthreads();
@@ -640,9 +628,9 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tmem_alloc(sTmem, 512);
     sm100::tmem_relinquish();
   }
-  stage_kmajor<D>(sBr, p.rot16, D);
-  stage_kmajor<D>(sBr + D * D * 2, p.rot16 + (size_t)D * D, D);
-  if constexpr (QJL) stage_kmajor<D>(sBs, p.s16, D);
+  sm100::stage_kmajor<D>(sBr, p.rot16, D);
+  sm100::stage_kmajor<D>(sBr + D * D * 2, p.rot16 + (size_t)D * D, D);
+  if constexpr (QJL) sm100::stage_kmajor<D>(sBs, p.s16, D);
   sm100::fence_proxy_async();
   sm100::tc_fence_before();
   __syncthreads();
@@ -1041,9 +1029,9 @@ k_encode_pp(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tmem_alloc(sTmem, kCols);
     sm100::tmem_relinquish();
   }
-  stage_kmajor<D>(sBr, p.rot16, D);
-  stage_kmajor<D>(sBr + D * D * 2, p.rot16 + (size_t)D * D, D);
-  stage_kmajor<D>(sBs, p.s16, D);
+  sm100::stage_kmajor<D>(sBr, p.rot16, D);
+  sm100::stage_kmajor<D>(sBr + D * D * 2, p.rot16 + (size_t)D * D, D);
+  sm100::stage_kmajor<D>(sBs, p.s16, D);
   sm100::fence_proxy_async();
   sm100::tc_fence_before();
   __syncthreads();

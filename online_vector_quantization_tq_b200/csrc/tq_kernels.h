@@ -61,6 +61,12 @@ tq_status dense_topk(const tq_quantizer *q, const float *ytil, const float *p, i
 tq_status rerank_launch(const float *y, int64_t nq, int64_t ldy, const void *x, bool bf16, int64_t n, int64_t ldx,
                         int d, const int64_t *cand, int kc, int k, float *out_s, int64_t *out_i, cudaStream_t st);
 
+// fp32 (or gathered) rows, Hadamard d in {32, 64, 128}: rotation on the CUDA
+// cores, QJL projection on the tensor cores.
+bool fwht_tc_encode_supported(const tq_quantizer *q);
+tq_status fwht_tc_encode(const tq_quantizer *q, const RowSource &src, int64_t n, void *codes, void *signs,
+                         float *norms, int64_t out_stride, cudaStream_t st);
+
 bool tc_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather);
 tq_status tc_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,
                     int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,

@@ -157,15 +157,21 @@ k_prep_operand(KernelTables kt, RowSource src, int64_t G, int N, int cexp, int8_
   x *= 1.0f / (float(D) * sqrtf(float(D)));
   v[j] = x;
   __syncthreads();
-  float acc0 = 0.f, acc1 = 0.f;
+  // p_j = sum_k S[j][k] y~_k: thread j reads row j of S with independent
+  // 16-byte loads (one L2 round trip), four partial sums over k mod 4
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
   if (kt.m > 0) {  // TurboQuant-MSE quantizers have no QJL projection (p = 0)
-#pragma unroll 8
-    for (int k = 0; k < D; k += 2) {
-      acc0 = fmaf(kt.qjl32t[(size_t)k * D + j], v[k], acc0);
-      acc1 = fmaf(kt.qjl32t[(size_t)(k + 1) * D + j], v[k + 1], acc1);
+    const float4 *srow = reinterpret_cast<const float4 *>(kt.qjl32 + (size_t)j * D);
+#pragma unroll
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      const float4 s4 = __ldg(srow + k4);
+      acc0 = fmaf(s4.x, v[4 * k4], acc0);
+      acc1 = fmaf(s4.y, v[4 * k4 + 1], acc1);
+      acc2 = fmaf(s4.z, v[4 * k4 + 2], acc2);
+      acc3 = fmaf(s4.w, v[4 * k4 + 3], acc3);
     }
   }
-  const float pj = acc0 + acc1;
+  const float pj = (acc0 + acc1) + (acc2 + acc3);
   // largest |y~| and |p|: power-of-two scales of the 16-bit fixed point
   float ay = fabsf(x), ap = fabsf(pj);
 #pragma unroll

@@ -305,6 +305,20 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return (uint32_t)row * 128u + (uint32_t)((chunk ^ (row & 7)) << 4);
 }
 
+// Copy a row-major 16-bit [rows][D] matrix from global memory into a 64-byte
+// swizzled K-major operand (D/32 blocks of rows x 64 B), all threads of the
+// block taking 16-byte chunks in turn.
+template <int D>
+__device__ void stage_kmajor(uint8_t *dst, const uint16_t *src, int rows) {
+  const int chunks = rows * (D / 8);
+  for (int i = threadIdx.x; i < chunks; i += blockDim.x) {
+    const int r = i / (D / 8), c8 = i % (D / 8);  // 8-element chunk index along K
+    const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * D + c8 * 8);
+    const int blk = c8 / 4, ch = c8 % 4;
+    *reinterpret_cast<uint4 *>(dst + (size_t)blk * rows * 64 + sw64_offset(r, ch)) = v;
+  }
+}
+
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

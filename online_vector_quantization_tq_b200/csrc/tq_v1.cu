@@ -260,15 +260,20 @@ k_prep_fwht_block(KernelTables kt, RowSource src, int64_t nq, float *ytil, float
   ytil[row * D + j] = x;
   if (kt.m == 0) return;  // TurboQuant-MSE: no QJL projection (uniform over the block)
   __syncthreads();
-  // p_j = sum_k S[j][k] y~_k: thread j walks column j of S^T, so every load
-  // of the warp is one contiguous segment
-  float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-  for (int k = 0; k < D; k += 2) {
-    acc0 = fmaf(kt.qjl32t[(size_t)k * D + j], v[k], acc0);
-    acc1 = fmaf(kt.qjl32t[(size_t)(k + 1) * D + j], v[k + 1], acc1);
+  // p_j = sum_k S[j][k] y~_k: thread j reads row j of S with independent
+  // 16-byte loads (one L2 round trip), four partial sums over k mod 4 (the
+  // same order as the integer scorer's fused query preparation)
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  const float4 *srow = reinterpret_cast<const float4 *>(kt.qjl32 + (size_t)j * D);
+#pragma unroll
+  for (int k4 = 0; k4 < D / 4; ++k4) {
+    const float4 s4 = __ldg(srow + k4);
+    acc0 = fmaf(s4.x, v[4 * k4], acc0);
+    acc1 = fmaf(s4.y, v[4 * k4 + 1], acc1);
+    acc2 = fmaf(s4.z, v[4 * k4 + 2], acc2);
+    acc3 = fmaf(s4.w, v[4 * k4 + 3], acc3);
   }
-  p[row * D + j] = acc0 + acc1;
+  p[row * D + j] = (acc0 + acc1) + (acc2 + acc3);
 }
 
 // Dense rotation, d <= 128: one block per query; y~ = R y walks the
