@@ -951,311 +951,6 @@ tq_status launch_tc2(const void *x, int64_t n, int64_t ldx, const EncTCParams &p
 }
 }  // namespace
 
-// ============================================================================
-// Encode for bf16 keys with the Hadamard rotation, two tile pipelines per CTA.
-//
-// The CTA holds the rotation K = d^1.5 R (two exact bf16 pieces) and S once
-// in shared memory and runs two independent pipelines of 256 threads over
-// alternate tiles of 128 keys.  Each pipeline owns one x tile buffer and 2d
-// TMEM columns (U, then Z):
-//
-//   TMA   x tile -> shared memory (the MMA's A operand as loaded)
-//   MMA   U = X K^T (bf16, two pieces) into TMEM
-//   ALU   ||U|| (two threads per row), codes, residual r = u - c[code];
-//         r is written back into U's own columns as fp16 hi + lo pieces
-//   MMA   Z = [r_hi | r_lo] S^T with the A operand read from TMEM
-//   ALU   sign bits of Z, norms
-//
-// While one pipeline waits for its tensor-core work the other computes, so
-// the CUDA-core and tensor-core phases of neighbouring tiles overlap without
-// a CTA-wide barrier.  Method: TurboQuant article 1.2.1-1.2.3 (rotation,
-// Lloyd-Max code, residual, QJL sign sketch), 2.1 (structured rotation),
-// 4.2.1 (stored norm).
-// ============================================================================
-namespace {
-
-template <int D>
-struct EncPPSmem {
-  static constexpr int kXBytes = kRows * D * 2;          // one bf16 tile (TMA, 128-byte swizzle)
-  static constexpr int kOffX = 0;                        // pipeline 0's tile, then pipeline 1's
-  static constexpr int kOffBr = 2 * kXBytes;             // K_hi, K_lo (bf16, 64-byte swizzle)
-  static constexpr int kOffBs = kOffBr + 2 * D * D * 2;  // S (fp16)
-  static constexpr int kOffPart = kOffBs + D * D * 2;    // row partial sums [pipe][kind][half][row]
-  static constexpr int kOffMisc = kOffPart + 2 * 2 * 2 * kRows * 4;
-  static constexpr int kTotal = kOffMisc + 256 + 1024;   // + alignment slack
-};
-
-}  // namespace
-
-template <int D, int W>
-__global__ void __launch_bounds__(512, 1)
-k_encode_pp(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
-  constexpr int L = 1 << W;
-  constexpr int HALF = L / 2;
-  constexpr int NB = D / 64;      // TMA boxes of 64 columns per tile
-  constexpr int CPT = D / 64;     // 32-coordinate chunks per thread (two threads per row)
-  constexpr int kPipe = 256;      // threads per pipeline
-  constexpr uint32_t kCols = 4 * D;
-  using SM = EncPPSmem<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sBr = smem + SM::kOffBr;
-  uint8_t *sBs = smem + SM::kOffBs;
-  float *sPart = reinterpret_cast<float *>(smem + SM::kOffPart);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffMisc);  // per pipeline: full, rot, qjl, drain
-  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 8);
-  volatile int *sAbort = reinterpret_cast<volatile int *>(sTmem + 2);  // one flag per pipeline
-
-  const int tid = threadIdx.x;
-  const int pp = tid >> 8;           // pipeline
-  const int t = tid & (kPipe - 1);
-  const int wq = (t >> 5) & 3;       // TMEM lane quadrant of this warp
-  const int h = t >> 7;              // half of the row's coordinates this thread owns
-  const int row = wq * 32 + (t & 31);
-  const uint32_t lane = (uint32_t)(wq * 32) << 16;
-  const bool issuer = t == 0;
-  uint64_t *bar_full = bars + 4 * pp, *bar_rot = bar_full + 1, *bar_qjl = bar_full + 2, *bar_drain = bar_full + 3;
-  uint8_t *sX = smem + SM::kOffX + pp * SM::kXBytes;
-  auto part = [&](int kind, int half, int r) -> float & { return sPart[((pp * 2 + kind) * 2 + half) * kRows + r]; };
-
-  if (tid == 0) {
-    for (int i = 0; i < 8; ++i) sm100::mbar_init(&bars[i], 1);
-    sm100::fence_barrier_init();
-    sm100::prefetch_tmap(&xmap);
-    sAbort[0] = 0;
-    sAbort[1] = 0;
-  }
-  if (tid < 32) {
-    sm100::tmem_alloc(sTmem, kCols);
-    sm100::tmem_relinquish();
-  }
-  sm100::stage_kmajor<D>(sBr, p.rot16, D);
-  sm100::stage_kmajor<D>(sBr + D * D * 2, p.rot16 + (size_t)D * D, D);
-  sm100::stage_kmajor<D>(sBs, p.s16, D);
-  sm100::fence_proxy_async();
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
-  const uint32_t tU = *sTmem + (uint32_t)(pp * 2 * D);
-  const uint32_t tZ = tU + D;
-
-  // symmetric codebook, scaled 2^10 (as in k_encode_tc2): magnitude
-  // thresholds as exact saturated steps on u^2, centroid magnitude steps
-  constexpr float kBig = 1099511627776.0f;  // 2^40
-  float nT2B[HALF], ndC[HALF];
-#pragma unroll
-  for (int k = 0; k < HALF; ++k) {
-    const float tk = p.thr_s[HALF - 1 + k];
-    nT2B[k] = -(tk * tk) * kBig;
-    ndC[k] = -(k == 0 ? p.cen_s[HALF] : p.cen_s[HALF + k] - p.cen_s[HALF + k - 1]);
-  }
-
-  const uint32_t idesc_rot = sm100::idesc_bf16_f32(kRows, D);
-  const uint32_t idesc_qjl = sm100::idesc_f16_f32(kRows, D);
-  const int first = blockIdx.x, stride = gridDim.x;
-  const int nloc = first < p.ntiles ? (p.ntiles - first + stride - 1) / stride : 0;
-  const int nit = nloc > pp ? (nloc - pp + 1) / 2 : 0;  // this pipeline's tiles: local indices pp, pp+2, ...
-  auto tile_of = [&](int it) { return first + (pp + 2 * it) * stride; };
-
-  auto issue_tma = [&](int tile) {
-    sm100::mbar_expect_tx(bar_full, SM::kXBytes);
-#pragma unroll
-    for (int bx = 0; bx < NB; ++bx)
-      sm100::tma_load_2d(sX + bx * (kRows * 128), &xmap, bx * 64, tile * kRows, bar_full);
-  };
-  auto issue_rot = [&]() {
-    const uint32_t xa = sm100::smem_u32(sX), br = sm100::smem_u32(sBr);
-#pragma unroll
-    for (int piece = 0; piece < 2; ++piece)
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint64_t a = sm100::desc_sw128(xa + (ks >> 2) * (kRows * 128) + (ks & 3) * 32);
-        const uint64_t b = sm100::desc_sw64(br + piece * (D * D * 2) + (ks >> 1) * (D * 64) + (ks & 1) * 32);
-        sm100::mma_f16(tU, a, b, idesc_rot, (piece | ks) != 0);
-      }
-    sm100::mma_commit(bar_rot);
-  };
-  // K order of the residual operand in TMEM: per 32-coordinate chunk c, 16
-  // columns of hi pairs then 16 of lo pairs, so K-step ks reads columns
-  // [8 ks, 8 ks + 8) and pairs with S's coordinates 32 (ks/4) + 16 (ks%2).
-  auto issue_qjl = [&]() {
-    const uint32_t bs = sm100::smem_u32(sBs);
-#pragma unroll
-    for (int ks = 0; ks < 2 * D / 16; ++ks) {
-      const uint64_t b = sm100::desc_sw64(bs + (ks >> 2) * (D * 64) + (ks & 1) * 32);
-      sm100::mma_f16_ts(tZ, tU + 8u * ks, b, idesc_qjl, ks != 0);
-    }
-    sm100::mma_commit(bar_qjl);
-  };
-
-  bool pend_tma = false;
-  uint32_t pend_par = 0u, ph = 0u;
-  if (issuer && nit > 0) {
-    issue_tma(tile_of(0));
-    pend_tma = true;
-  }
-  const float2 big2 = make_float2(kBig, kBig);
-  const float2 base2 = make_float2(8388608.0f + (float)HALF, 8388608.0f + (float)HALF);
-  bool failed = false;  // pipeline-uniform: only set from a barrier vote
-  for (int it = 0; it < nit; ++it) {
-    const int64_t grow = (int64_t)tile_of(it) * kRows + row;
-    bool ok = true;
-    // ---- rotation
-    if (issuer) {
-      ok = sm100::mbar_wait_abort(bar_full, ph, sAbort + pp, p.err, 21);
-      if (ok) {
-        pend_tma = false;
-        sm100::tc_fence_after();
-        issue_rot();
-      }
-    }
-    ok = sm100::mbar_wait_abort(bar_rot, ph, sAbort + pp, p.err, 22) && ok;
-    if (issuer && ok && it + 1 < nit) {  // the rotation has read the tile: load the next one
-      issue_tma(tile_of(it + 1));
-      pend_tma = true;
-      pend_par = ph ^ 1u;
-    }
-    sm100::tc_fence_after();
-    // ---- ||U||^2 of this thread's half row
-    {
-      float2 ss = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < CPT; ++k) {
-        uint32_t u[32];
-        sm100::tmem_ld32(tU + lane + 32 * (h * CPT + k), u);
-        sm100::tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 v = make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1]));
-          ss = __ffma2_rn(v, v, ss);
-        }
-      }
-      part(0, h, row) = ss.x + ss.y;
-    }
-    failed = sm100::named_barrier_or(1 + pp, kPipe, !ok);
-    if (failed) break;
-    // ---- codes and residual
-    const float nacc = sqrtf(part(0, 0, row) + part(0, 1, row));
-    const float nrm = nacc * p.rho;
-    const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;  // zero rows: u = -0 -> lower middle code
-    const float2 sv2 = make_float2(s_v, s_v);
-    float2 g2 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < CPT; ++k) {
-      const int c = h * CPT + k;
-      uint32_t acc[32];
-      sm100::tmem_ld32(tU + lane + 32 * c, acc);
-      sm100::tmem_wait_ld();
-      RawPack<W> pk;
-      uint32_t rv[32];  // residual operand: 16 hi pairs, then 16 lo pairs
-#pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 us = __fmul2_rn(make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])), sv2);
-        const float2 usb = __fmul2_rn(us, big2);
-        float2 ncm = make_float2(ndC[0], ndC[0]), mh = make_float2(0.5f, 0.5f);
-#pragma unroll
-        for (int q = 1; q < HALF; ++q) {
-          const float2 st = make_float2(__saturatef(__fmaf_rn(us.x, usb.x, nT2B[q])),
-                                        __saturatef(__fmaf_rn(us.y, usb.y, nT2B[q])));
-          ncm = __ffma2_rn(st, make_float2(ndC[q], ndC[q]), ncm);
-          mh = __fadd2_rn(mh, st);
-        }
-        const float2 sg = make_float2(__uint_as_float((__float_as_uint(us.x) & 0x80000000u) | 0x3F800000u),
-                                      __uint_as_float((__float_as_uint(us.y) & 0x80000000u) | 0x3F800000u));
-        const float2 codef = ffma2_rm(sg, mh, base2);  // 2^23 + code, exactly
-        const float2 rr = __ffma2_rn(sg, ncm, us);     // u - c[code]
-        pk.add(j, __float_as_uint(codef.x));
-        pk.add(j + 1, __float_as_uint(codef.y));
-        g2 = __ffma2_rn(rr, rr, g2);
-        const __half2 hh = __floats2half2_rn(rr.x, rr.y);
-        const float2 hf = __half22float2(hh);
-        rv[j / 2] = *reinterpret_cast<const uint32_t *>(&hh);
-        const float2 lf = __fadd2_rn(rr, make_float2(-hf.x, -hf.y));
-        rv[16 + j / 2] = pack_half2(lf.x, lf.y);
-      }
-      sm100::tmem_st32(tU + lane + 32 * c, rv);
-      uint32_t cw[W];
-      pk.finish(cw);
-      if (grow < p.n) {
-        uint32_t *dst = p.codes + grow * p.out_stride * (W * D / 32) + c * W;
-#pragma unroll
-        for (int q = 0; q < W; ++q) dst[q] = cw[q];
-      }
-    }
-    sm100::tmem_wait_st();
-    part(1, h, row) = g2.x + g2.y;
-    sm100::tc_fence_before();
-    sm100::named_barrier(1 + pp, kPipe);
-    // ---- QJL projection and sign bits
-    if (issuer) {
-      sm100::tc_fence_after();
-      issue_qjl();
-    }
-    ok = sm100::mbar_wait_abort(bar_qjl, ph, sAbort + pp, p.err, 23);
-    sm100::tc_fence_after();
-#pragma unroll
-    for (int k = 0; k < CPT; ++k) {
-      const int c = h * CPT + k;
-      uint32_t z[32];
-      sm100::tmem_ld32(tZ + lane + 32 * c, z);
-      sm100::tmem_wait_ld();
-      uint32_t wbits = 0u;
-#pragma unroll
-      for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
-      if (ok && grow < p.n) p.signs[grow * p.out_stride * (D / 32) + c] = ~wbits;
-    }
-    if (ok && h == 0 && grow < p.n) {
-      const float gam = sqrtf(part(1, 0, row) + part(1, 1, row)) * (1.0f / kRScale);
-      p.norms[grow * p.out_stride] = make_float2(nrm, gam);
-    }
-    ph ^= 1u;
-    sm100::tc_fence_before();
-    failed = sm100::named_barrier_or(1 + pp, kPipe, !ok);
-    if (failed) break;
-  }
-  if (failed && issuer) {
-    if (pend_tma) sm100::mbar_wait(bar_full, pend_par, p.err, 24);  // a load still in flight
-    // MMAs issued may still run: wait (bounded) before TMEM is freed
-    sm100::mma_commit(bar_drain);
-    sm100::mbar_wait(bar_drain, 0u, p.err, 25);
-  }
-  sm100::tc_fence_before();
-  __syncthreads();
-  if (tid < 32) sm100::tmem_dealloc(*sTmem, kCols);
-}
-
-namespace {
-template <int D, int W>
-tq_status launch_pp(const void *x, int64_t n, int64_t ldx, const EncTCParams &prm, cudaStream_t st) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return TQ_ERR_CUDA;
-  CUtensorMap map;
-  cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)n};
-  cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), gdim, gstride, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return TQ_ERR_CUDA;
-  int dev = 0, max_smem = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // at least half the SM's shared memory, so that one CTA (which allocates
-  // TMEM for both pipelines) runs per SM
-  const int smem = std::max(EncPPSmem<D>::kTotal, max_smem / 2 + 1024);
-  if (smem > max_smem) return TQ_ERR_UNSUPPORTED;
-  EncTCParams pp = prm;
-  pp.ntiles = (int)((n + kRows - 1) / kRows);
-  auto kern = k_encode_pp<D, W>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return TQ_ERR_CUDA;
-  kern<<<std::min(pp.ntiles, sms), 512, smem, st>>>(map, pp);
-  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
-}
-}  // namespace
-
 bool tc2_encode_supported(const tq_quantizer *q, int dtype, bool gather) {
   return dtype == TQ_BF16 && !gather && q->d_rot_bf16 && (q->d == 64 || q->d == 128);
 }

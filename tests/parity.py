@@ -57,8 +57,14 @@ def check_encode(codes_u8, signs_u8, norms, x, t: "o.Tables", ref=None) -> Encod
 
 
 def score_errors(s_gpu, s_ref, xnorm, ynorm, d, skip_keys=None):
+    """Relative score errors against max(|s|, ||x|| ||y|| / sqrt(d)); where
+    that is 0 (a zero key or query, whose score is exactly 0), the GPU score
+    must be exactly 0 too (error 0, else inf)."""
     floor = np.outer(ynorm, xnorm) / math.sqrt(d)
-    err = np.abs(s_gpu.astype(np.float64) - s_ref) / np.maximum(np.abs(s_ref), floor)
+    diff = np.abs(s_gpu.astype(np.float64) - s_ref)
+    den = np.maximum(np.abs(s_ref), floor)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        err = np.where(den > 0, diff / np.where(den > 0, den, 1.0), np.where(diff == 0, 0.0, np.inf))
     if skip_keys is not None and np.any(skip_keys):
         err[:, skip_keys] = 0.0
     return err
