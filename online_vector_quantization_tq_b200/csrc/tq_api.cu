@@ -82,6 +82,8 @@ tq_status tq_encode_ws(const tq_quantizer *q, const void *x, tq_dtype dtype, int
   }
   if (tc2_encode_supported(q, dtype, chan != nullptr))
     return tc2_encode(q, x, n, ldx, codes, signs, norms, out_stride, s);
+  if (tcg_encode_supported(q, dtype, ldx, chan != nullptr))
+    return tcg_encode(q, x, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, s);
   if (tc_encode_supported(q, dtype, ldx, chan != nullptr))
     return tc_encode(q, x, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, s);
   if (fwht_tc_encode_supported(q)) return fwht_tc_encode(q, src, n, codes, signs, norms, out_stride, s);

@@ -921,6 +921,451 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   if (tid < 32) sm100::tmem_dealloc(tmem, 512);
 }
 
+// ============================================================================
+// Encode of bf16 keys whose coordinates are gathered through a per-group
+// channel map (the 3.5- and 2.5-bit outlier splits of the KV cache,
+// TurboQuant article 4.1.1), d in {32, 64, 96}, Hadamard or Haar rotation.
+// The structure of k_encode_tc2 (16-coordinate-group compute warps, a
+// control warp issuing every TMA load and MMA, U double-buffered in TMEM,
+// the rotation two tiles ahead), with one more step: the compute threads
+// gather a tile's channels from the raw TMA tile into the rotation's A
+// operand (bf16, exact), two tiles ahead of its rotation.  The rotation's B
+// operand is RP exact bf16 pieces: d^1.5 R (an integer matrix, two pieces)
+// for Hadamard, the fp32 Haar matrix (three pieces) for Haar.
+// ============================================================================
+namespace {
+
+template <int D, int RP, int SRCW>
+struct EncGSmem {
+  static constexpr int kXBytes = kRows * SRCW * 2;           // the raw bf16 tile (TMA, 128-byte swizzle)
+  static constexpr int kAxBytes = kRows * D * 2;             // one gathered A operand (64-byte swizzle)
+  static constexpr int kOffX = 0;
+  static constexpr int kOffAx = kOffX + kXBytes;             // two of them
+  static constexpr int kOffAr = kOffAx + 2 * kAxBytes;       // [r_hi | r_lo] fp16
+  static constexpr int kOffBr = kOffAr + kRows * 2 * D * 2;  // RP rotation pieces, bf16
+  static constexpr int kOffBs = kOffBr + RP * D * D * 2;     // S fp16
+  static constexpr int kOffMisc = kOffBs + D * D * 2;
+  static constexpr int kTotal = kOffMisc + 128 + 1024;
+};
+
+}  // namespace
+
+template <int D, int W, int RP, int SRCW>
+__global__ void __launch_bounds__(128 * (D / 32) + 32, 1)
+k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
+  constexpr int P = D / 32;
+  constexpr int L = 1 << W;
+  constexpr int HALF = L / 2;
+  constexpr int NB = SRCW / 64;      // TMA boxes of 64 columns
+  constexpr int kCompute = 128 * P;  // compute threads; one more warp issues the copies and MMAs
+  constexpr uint32_t kColU0 = 0, kColZ = 256, kColScr = 384;
+  using SM = EncGSmem<D, RP, SRCW>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sX = smem + SM::kOffX;
+  uint8_t *sAx = smem + SM::kOffAx;
+  uint8_t *sAr = smem + SM::kOffAr;
+  uint8_t *sBr = smem + SM::kOffBr;
+  uint8_t *sBs = smem + SM::kOffBs;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffMisc);  // full, rot, qjl, drain
+  uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
+
+  const int tid = threadIdx.x;
+  const bool compute = tid < kCompute;
+  const bool ctl = tid == kCompute;
+  const int row = tid & (kRows - 1);
+  const int pc = tid >> 7;
+  const uint32_t lane = (uint32_t)(row & ~31) << 16;
+
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) sm100::mbar_init(&bars[i], 1);
+    sm100::fence_barrier_init();
+    sm100::prefetch_tmap(&xmap);
+  }
+  if (tid < 32) {
+    sm100::tmem_alloc(sTmem, 512);
+    sm100::tmem_relinquish();
+  }
+#pragma unroll
+  for (int k = 0; k < RP; ++k) sm100::stage_kmajor<D>(sBr + k * (D * D * 2), p.rot16 + (size_t)k * D * D, D);
+  sm100::stage_kmajor<D>(sBs, p.s16, D);
+  sm100::fence_proxy_async();
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+
+  constexpr float kBig = 1099511627776.0f;  // 2^40: exact steps sat(2^40 (|u| - T_k))
+  float nTB[HALF], ndC[HALF];
+#pragma unroll
+  for (int k = 0; k < HALF; ++k) {
+    nTB[k] = -p.thr_s[HALF - 1 + k] * kBig;
+    ndC[k] = -(k == 0 ? p.cen_s[HALF] : p.cen_s[HALF + k] - p.cen_s[HALF + k - 1]);
+  }
+  const uint32_t idesc_rot = sm100::idesc_bf16_f32(kRows, D);
+  const uint32_t idesc_qjl = sm100::idesc_f16_f32(kRows, D);
+  const int first = blockIdx.x, stride = gridDim.x;
+  const int nloc = first < p.ntiles ? (p.ntiles - first + stride - 1) / stride : 0;
+
+  auto issue_tma = [&](int tile, int &count) {
+    sm100::mbar_expect_tx(&bars[0], SM::kXBytes);
+#pragma unroll
+    for (int bx = 0; bx < NB; ++bx)
+      sm100::tma_load_2d(sX + bx * (kRows * 128), &xmap, bx * 64, tile * kRows, &bars[0]);
+    ++count;
+  };
+  auto issue_rot = [&](int abuf, uint32_t ucol) {
+    const uint32_t xa = sm100::smem_u32(sAx + abuf * SM::kAxBytes), br = sm100::smem_u32(sBr);
+#pragma unroll
+    for (int piece = 0; piece < RP; ++piece)
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t a = sm100::desc_sw64(xa + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+        const uint64_t b = sm100::desc_sw64(br + piece * (D * D * 2) + (ks >> 1) * (D * 64) + (ks & 1) * 32);
+        sm100::mma_f16(tmem + ucol, a, b, idesc_rot, (piece | ks) != 0);
+      }
+    sm100::mma_commit(&bars[1]);
+  };
+  auto issue_qjl = [&]() {
+    const uint32_t ar = sm100::smem_u32(sAr), bs = sm100::smem_u32(sBs);
+#pragma unroll
+    for (int ks = 0; ks < 2 * D / 16; ++ks) {
+      const int kk = ks % (D / 16);
+      const uint64_t a = sm100::desc_sw64(ar + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+      const uint64_t b = sm100::desc_sw64(bs + (kk >> 1) * (D * 64) + (kk & 1) * 32);
+      sm100::mma_f16(tmem + kColZ, a, b, idesc_qjl, ks != 0);
+    }
+    sm100::mma_commit(&bars[2]);
+  };
+  // gather this thread's 32 channels of tile `tile` from the raw tile into A operand `abuf`
+  auto gather = [&](int tile, int abuf) {
+    const int64_t grow = (int64_t)tile * kRows + row;
+    const int32_t *ch = p.chan + (grow < p.n ? grow / p.chan_rows : 0) * D + 32 * pc;
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      // masked to the staged tile: a channel index cannot address beyond it
+      const int s0 = __ldg(ch + j) & (SRCW - 1), s1 = __ldg(ch + j + 1) & (SRCW - 1);
+      const uint32_t h0 = *reinterpret_cast<const uint16_t *>(sX + (s0 / 64) * (kRows * 128) +
+                                                              sm100::sw128_offset(row, (s0 % 64) / 8) + (s0 % 8) * 2);
+      const uint32_t h1 = *reinterpret_cast<const uint16_t *>(sX + (s1 / 64) * (kRows * 128) +
+                                                              sm100::sw128_offset(row, (s1 % 64) / 8) + (s1 % 8) * 2);
+      w[j / 2] = h0 | (h1 << 16);
+    }
+    uint8_t *dst = sAx + abuf * SM::kAxBytes + pc * (kRows * 64);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      *reinterpret_cast<uint4 *>(dst + sm100::sw64_offset(row, k)) =
+          make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    sm100::fence_proxy_async();
+  };
+  auto norm_col = [&](int par) { return (uint32_t)(kColScr + 16 * par); };
+  auto gam_col = [&](int par) { return (uint32_t)(kColScr + 16 * par + 8); };
+  auto row_partial = [&](uint32_t ucol, uint32_t scol) {
+    uint32_t u[32];
+    sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, u);
+    sm100::tmem_wait_ld();
+    float2 ss = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float2 v = make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1]));
+      ss = __ffma2_rn(v, v, ss);
+    }
+    sm100::tmem_st1(tmem + lane + scol + pc, __float_as_uint(ss.x + ss.y));
+  };
+  auto sum_parts = [&](uint32_t scol) {
+    uint32_t parts[4];
+    sm100::tmem_ld4(tmem + lane + scol, parts);
+    sm100::tmem_wait_ld();
+    float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < P; ++k) v += __uint_as_float(parts[k]);
+    return v;
+  };
+  auto sign_word = [&]() {
+    uint32_t z[32];
+    sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+    sm100::tmem_wait_ld();
+    uint32_t wbits = 0u;
+#pragma unroll
+    for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
+    return ~wbits;
+  };
+
+  uint32_t ph_full = 0u, ph_rot = 0u, ph_qjl = 0u;  // compute threads' phases
+  bool pend_full = false;  // control thread: a raw-tile load in flight, the ntma-th
+  int ntma = 0;
+  bool failed = false;     // CTA-uniform: only ever set from a barrier vote
+  bool ifail = false;
+  bool any_mma = false;
+  // compute threads: wait for raw tile `tile` and gather it into `abuf`
+  auto wait_and_gather = [&](int tile, int abuf) {
+    const bool ok = sm100::mbar_wait(&bars[0], ph_full, p.err, 61);
+    ph_full ^= 1u;
+    gather(tile, abuf);
+    return ok;
+  };
+
+  // ---- prologue: tiles 0 and 1 gathered and rotated, the norm parts of tile 0
+  if (nloc > 0) {
+    if (ctl) {
+      issue_tma(first, ntma);
+      pend_full = true;
+    }
+    bool ok = compute ? wait_and_gather(first, 0) : true;
+    failed = __syncthreads_or(!ok) != 0;
+    if (!failed) {
+      if (ctl) {
+        pend_full = false;
+        sm100::tc_fence_after();
+        issue_rot(0, kColU0);
+        any_mma = true;
+        if (nloc > 1) {
+          issue_tma(first + stride, ntma);
+          pend_full = true;
+        }
+      }
+      ok = (compute && nloc > 1) ? wait_and_gather(first + stride, 1) : true;
+      failed = __syncthreads_or(!ok) != 0;
+    }
+    if (!failed) {
+      if (ctl) {
+        pend_full = false;
+        sm100::tc_fence_after();
+        if (nloc > 1) issue_rot(1, 128u);
+        if (nloc > 2) {
+          issue_tma(first + 2 * stride, ntma);
+          pend_full = true;
+        }
+      }
+      ok = true;
+      if (compute) {
+        ok = sm100::mbar_wait(&bars[1], ph_rot, p.err, 62);
+        ph_rot ^= 1u;
+        sm100::tc_fence_after();
+        row_partial(kColU0, norm_col(0));
+        sm100::tmem_wait_st();
+      }
+      sm100::tc_fence_before();
+      failed = __syncthreads_or(!ok) != 0;
+      sm100::tc_fence_after();
+    }
+  }
+
+  float prev_norm = 0.f;
+  int64_t prev_row = -1;
+  const float2 base2 = make_float2(8388608.0f + (float)HALF, 8388608.0f + (float)HALF);
+  int it = 0;
+  for (; it < nloc && !failed; ++it) {
+    const int t = first + it * stride;
+    const int par = it & 1;
+    const uint32_t ucol = par ? 128u : 0u;
+    const int64_t grow = (int64_t)t * kRows + row;
+    bool ok = true;
+    if (compute) {
+      // ---- (a) codes and residual of this tile
+      const float nacc = sqrtf(sum_parts(norm_col(par)));
+      const float nrm = nacc * p.rho;
+      const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;
+      const float2 sv2 = make_float2(s_v, s_v);
+      uint32_t acc[32];
+      sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
+      sm100::tmem_wait_ld();
+      RawPack<W> pk;
+      uint32_t hi[16], lo[16];
+      float2 g2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float2 us = __fmul2_rn(make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])), sv2);
+        float2 ncm = make_float2(ndC[0], ndC[0]), mh = make_float2(0.5f, 0.5f);
+#pragma unroll
+        for (int k = 1; k < HALF; ++k) {
+          const float2 st = make_float2(__saturatef(__fmaf_rn(fabsf(us.x), kBig, nTB[k])),
+                                        __saturatef(__fmaf_rn(fabsf(us.y), kBig, nTB[k])));
+          ncm = __ffma2_rn(st, make_float2(ndC[k], ndC[k]), ncm);
+          mh = __fadd2_rn(mh, st);
+        }
+        const float2 sg = make_float2(__uint_as_float((__float_as_uint(us.x) & 0x80000000u) | 0x3F800000u),
+                                      __uint_as_float((__float_as_uint(us.y) & 0x80000000u) | 0x3F800000u));
+        const float2 codef = ffma2_rm(sg, mh, base2);
+        const float2 rr = __ffma2_rn(sg, ncm, us);
+        pk.add(j, __float_as_uint(codef.x));
+        pk.add(j + 1, __float_as_uint(codef.y));
+        g2 = __ffma2_rn(rr, rr, g2);
+        const __half2 h = __floats2half2_rn(rr.x, rr.y);
+        const float2 hf = __half22float2(h);
+        hi[j / 2] = *reinterpret_cast<const uint32_t *>(&h);
+        const float2 lf = __fadd2_rn(rr, make_float2(-hf.x, -hf.y));
+        lo[j / 2] = pack_half2(lf.x, lf.y);
+      }
+      uint32_t cw[W];
+      pk.finish(cw);
+      if (grow < p.n) {
+        uint32_t *dst = p.codes + grow * p.out_stride * (W * D / 32) + pc * W;
+#pragma unroll
+        for (int k = 0; k < W; ++k) dst[k] = cw[k];
+      }
+      // ---- (b) sign bits and norms of the previous tile
+      if (it > 0) {
+        ok = sm100::mbar_wait(&bars[2], ph_qjl, p.err, 63);
+        ph_qjl ^= 1u;
+        sm100::tc_fence_after();
+        const uint32_t sw = sign_word();
+        const float gam = pc == 0 ? sqrtf(sum_parts(gam_col(par ^ 1))) * (1.0f / kRScale) : 0.f;
+        if (prev_row >= 0 && prev_row < p.n) {
+          p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
+          if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
+        }
+      }
+      // ---- (c) residual operand
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        *reinterpret_cast<uint4 *>(sAr + pc * (kRows * 64) + sm100::sw64_offset(row, k)) =
+            make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
+        *reinterpret_cast<uint4 *>(sAr + (P + pc) * (kRows * 64) + sm100::sw64_offset(row, k)) =
+            make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+      }
+      // ---- (g) gather tile it+2 into this tile's A operand (its rotation is done)
+      if (it + 2 < nloc) ok = wait_and_gather(first + (it + 2) * stride, par) && ok;
+      // ---- (d) norm parts of the next tile, gamma parts of this one
+      if (it + 1 < nloc) {
+        ok = sm100::mbar_wait(&bars[1], ph_rot, p.err, 64) && ok;
+        ph_rot ^= 1u;
+        sm100::tc_fence_after();
+        row_partial(ucol ^ 128u, norm_col(par ^ 1));
+      }
+      sm100::tmem_st1(tmem + lane + gam_col(par) + pc, __float_as_uint(g2.x + g2.y));
+      sm100::tmem_wait_st();
+      sm100::fence_proxy_async();
+      prev_norm = nrm;
+      prev_row = grow;
+    }
+    sm100::tc_fence_before();
+    failed = __syncthreads_or(!ok || ifail) != 0;
+    if (failed) break;
+    sm100::tc_fence_after();
+    // ---- (e) control thread: QJL of this tile, the next raw tile, the rotation two tiles ahead
+    if (ctl) {
+      issue_qjl();
+      if (it + 2 < nloc) pend_full = false;  // consumed by the gather above
+      if (it + 3 < nloc) {
+        issue_tma(first + (it + 3) * stride, ntma);
+        pend_full = true;
+      }
+      if (it + 2 < nloc) issue_rot(par, ucol);
+    }
+  }
+
+  // ---- drain: sign bits and norms of the last tile
+  failed = __syncthreads_or(failed || ifail) != 0;
+  if (!failed && it > 0) {
+    const bool ok = __syncthreads_and(compute ? sm100::mbar_wait(&bars[2], ph_qjl, p.err, 65) : true) != 0;
+    sm100::tc_fence_after();
+    if (ok && compute) {
+      const uint32_t sw = sign_word();
+      const float gam = pc == 0 ? sqrtf(sum_parts(gam_col((it - 1) & 1))) * (1.0f / kRScale) : 0.f;
+      if (prev_row >= 0 && prev_row < p.n) {
+        p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
+        if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
+      }
+    }
+  }
+  if (failed && ctl) {
+    if (pend_full) sm100::mbar_wait(&bars[0], (uint32_t)((ntma - 1) & 1), p.err, 66);
+    if (any_mma) {
+      sm100::mma_commit(&bars[3]);
+      sm100::mbar_wait(&bars[3], 0u, p.err, 67);
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (tid < 32) sm100::tmem_dealloc(tmem, 512);
+}
+
+namespace {
+template <int D, int W, int RP>
+tq_status launch_tcg(const void *x, int64_t n, int64_t ldx, const EncTCParams &prm, cudaStream_t st) {
+  constexpr int SRCW = 128;
+  auto enc = tensor_map_encoder();
+  if (!enc) return TQ_ERR_CUDA;
+  CUtensorMap map;
+  cuuint64_t gdim[2] = {(cuuint64_t)ldx, (cuuint64_t)n};
+  cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), gdim, gstride, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return TQ_ERR_CUDA;
+  int dev = 0, max_smem = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // at least half the SM's shared memory, so that one CTA (which takes all of
+  // TMEM) runs per SM
+  const int smem = std::max(EncGSmem<D, RP, SRCW>::kTotal, max_smem / 2 + 1024);
+  if (smem > max_smem) return TQ_ERR_UNSUPPORTED;
+  EncTCParams pp = prm;
+  pp.ntiles = (int)((n + kRows - 1) / kRows);
+  auto kern = k_encode_tcg<D, W, RP, SRCW>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32) + 32, smem, st>>>(map, pp);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+template <int D, int RP>
+tq_status dispatch_tcg_w(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const EncTCParams &prm,
+                         cudaStream_t st) {
+  switch (q->w) {
+    case 1: return launch_tcg<D, 1, RP>(x, n, ldx, prm, st);
+    case 2: return launch_tcg<D, 2, RP>(x, n, ldx, prm, st);
+    case 3: return launch_tcg<D, 3, RP>(x, n, ldx, prm, st);
+    case 4: return launch_tcg<D, 4, RP>(x, n, ldx, prm, st);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+}  // namespace
+
+bool tcg_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather) {
+  if (dtype != TQ_BF16 || !gather || q->m != q->d || ldx != 128) return false;
+  if (q->rotation == TQ_ROT_HADAMARD) return q->d_rot_bf16 && (q->d == 32 || q->d == 64);
+  return q->d_rot_bf16x3 && (q->d == 32 || q->d == 64 || q->d == 96);
+}
+
+tq_status tcg_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,
+                     int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,
+                     cudaStream_t st) {
+  EncTCParams prm{};
+  prm.n = n;
+  const bool had = q->rotation == TQ_ROT_HADAMARD;
+  prm.rot16 = had ? q->d_rot_bf16 : q->d_rot_bf16x3;
+  prm.s16 = q->d_qjl16;
+  prm.rho = had ? q->tc_rho : 1.0f;  // U = d^1.5 R x (Hadamard) or R x (Haar)
+  for (int i = 0; i < kMaxLevels; ++i) {
+    prm.thr_s[i] = q->kt.thresholds[i] * kRScale;
+    prm.cen_s[i] = q->kt.centroids[i] * kRScale;
+  }
+  prm.chan = chan;
+  prm.chan_rows = chan_rows;
+  prm.codes = static_cast<uint32_t *>(codes);
+  prm.signs = static_cast<uint32_t *>(signs);
+  prm.norms = reinterpret_cast<float2 *>(norms);
+  prm.out_stride = out_stride;
+  prm.err = q->d_err;
+  if (had) {
+    if (q->d == 32) return dispatch_tcg_w<32, 2>(q, x, n, ldx, prm, st);
+    if (q->d == 64) return dispatch_tcg_w<64, 2>(q, x, n, ldx, prm, st);
+    return TQ_ERR_UNSUPPORTED;
+  }
+  switch (q->d) {
+    case 32: return dispatch_tcg_w<32, 3>(q, x, n, ldx, prm, st);
+    case 64: return dispatch_tcg_w<64, 3>(q, x, n, ldx, prm, st);
+    case 96: return dispatch_tcg_w<96, 3>(q, x, n, ldx, prm, st);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
 namespace {
 template <int D, int W, bool QJL>
 tq_status launch_tc2(const void *x, int64_t n, int64_t ldx, const EncTCParams &prm, cudaStream_t st) {

@@ -282,6 +282,8 @@ void free_device(tq_quantizer *q) {
   q->d_qjl_limbs = nullptr;
   cudaFree(q->d_rot16);
   cudaFree(q->d_rot_bf16);
+  cudaFree(q->d_rot_bf16x3);
+  q->d_rot_bf16x3 = nullptr;
   cudaFree(q->d_err);
   q->d_rot16 = nullptr;
   q->d_rot_bf16 = nullptr;
@@ -510,6 +512,34 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
         st = upload(&q->d_rot_bf16, bfp.data(), bfp.size());
       }
     } else {
+      if (d <= 128) {
+        // the fp32 R as three bf16 pieces (8 + 8 + 8 significant bits: exact),
+        // for the gathered tensor-core encode of bf16 keys
+        std::vector<uint16_t> b3(3 * dd);
+        auto bf = [](float f) {
+          uint32_t b;
+          std::memcpy(&b, &f, 4);
+          b += 0x7FFFu + ((b >> 16) & 1u);
+          return (uint16_t)(b >> 16);
+        };
+        auto fb = [](uint16_t h) {
+          uint32_t b = (uint32_t)h << 16;
+          float f;
+          std::memcpy(&f, &b, 4);
+          return f;
+        };
+        for (size_t i = 0; i < dd; ++i) {
+          const float r0 = q->rot[i];
+          const uint16_t h0 = bf(r0);
+          const float r1 = r0 - fb(h0);  // exact: fewer significant bits than r0
+          const uint16_t h1 = bf(r1);
+          const float r2 = r1 - fb(h1);
+          b3[i] = h0;
+          b3[dd + i] = h1;
+          b3[2 * dd + i] = bf(r2);
+        }
+        st = upload(&q->d_rot_bf16x3, b3.data(), b3.size());
+      }
       q->tc_rho = 1.0f / 256.0f;
       q->tc_rot_pieces = 2;
       pieces.resize(2 * dd);

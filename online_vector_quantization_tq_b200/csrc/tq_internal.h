@@ -49,6 +49,7 @@ struct tq_quantizer {
   int tc_rot_pieces = 0;
   float tc_rho = 0.f;
   uint16_t *d_rot_bf16 = nullptr;  // Hadamard: d^1.5 R as two exact bf16 pieces [2][d][d]
+  uint16_t *d_rot_bf16x3 = nullptr;  // Haar (d <= 128): the fp32 R as three exact bf16 pieces [3][d][d]
   // dense tensor-core encode (d >= 256): R and S as 31-bit fixed point,
   // v 2^e = 2^24 a + 2^16 b + 2^8 c + d with signed bytes, stored as four
   // planes [4][rows][d] (a, b, c, d)

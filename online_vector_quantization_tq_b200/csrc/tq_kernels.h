@@ -72,6 +72,13 @@ tq_status tc_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx
                     int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,
                     cudaStream_t st);
 
+// Gathered bf16 rows (per-group channel map), d in {32, 64, 96}, Hadamard or
+// Haar: the tc2 structure with a gather step.
+bool tcg_encode_supported(const tq_quantizer *q, int dtype, int64_t ldx, bool gather);
+tq_status tcg_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, const int32_t *chan,
+                     int64_t chan_rows, void *codes, void *signs, float *norms, int64_t out_stride,
+                     cudaStream_t st);
+
 bool tc2_encode_supported(const tq_quantizer *q, int dtype, bool gather);
 tq_status tc2_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, void *codes, void *signs,
                      float *norms, int64_t out_stride, cudaStream_t st);

@@ -540,3 +540,28 @@ def test_two_stage_retrieval_recall(tq):
     r2 = np.mean([len(set(a) & set(b)) / 10 for a, b in zip(i2.cpu().numpy(), truth)])
     print(f"two-stage: recall@10 first stage {r1:.3f}, after re-scoring the top-64 {r2:.3f}")
     assert r2 >= r1 and r2 >= 0.97
+
+
+@pytest.mark.parametrize("d,b,rot", [(96, 2, "haar"), (32, 4, "hadamard"), (64, 3, "hadamard"), (64, 3, "haar")])
+def test_gathered_bf16_encode(tq, d, b, rot):
+    """bf16 rows of 128 channels encoded through a per-group channel map (the
+    outlier split's path): 1000 rows in groups of 300 (group boundaries
+    inside tiles, a ragged last tile), a zero row, codes and signs against
+    the oracle on the gathered channels, scores with the same map."""
+    rng = np.random.default_rng(d * 3 + b)
+    n, rows_per_group = 1000, 300
+    groups = (n + rows_per_group - 1) // rows_per_group
+    x = wl.to_bf16_values(rng.standard_normal((n, 128)).astype(np.float32) * rng.choice([1.0, 7.0], size=128))
+    x[11] = 0.0
+    chan = np.stack([np.sort(rng.permutation(128)[:d]) for _ in range(groups)]).astype(np.int32)
+    xg = np.stack([x[r, chan[r // rows_per_group]] for r in range(n)])
+    t = tables(d, b, rot)
+    q = tq.tq_codebook(d, b, seed=0, rotation=rot)
+    enc = tq.tq_encode(q, dev(x, torch.bfloat16), chan=dev(chan, torch.int32), chan_rows=rows_per_group)
+    rep = check_encode(*host(enc), xg, t)
+    y = rng.standard_normal((3, d)).astype(np.float32)
+    s = tq.tq_score(q, dev(y), 1, 3, enc, n).cpu().numpy()
+    skip = rep.skip_rows.copy()
+    check_scores(s, o.score(*o.prepare_query(y, t), rep.ref, t), rep.ref["norm"], np.linalg.norm(y, axis=1), d,
+                 skip)
+    assert np.all(s[:, 11] == 0.0)
