@@ -691,7 +691,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
                "encode_vectors_per_s": n / (enc_ms * 1e-3), "score_keys_per_s": n / (pm["score"] * 1e-3),
                "bytes_per_key": key_b,
                "l2": "two code buffers; each step scores the codes encoded one step earlier",
-               "roofline": {"encode": roofline_hbm(n * (256 + key_b), enc_ms, peak, "k_encode_tc",
+               "roofline": {"encode": roofline_hbm(n * (256 + key_b), enc_ms, peak, "k_encode_tcg",
                                                    f"{256 + key_b} B/key (256 in, {key_b} out), both parts"),
                             "score": roofline_hbm(n * (key_b + 16), pm["score"], peak, "k_score_tc",
                                                   f"{key_b + 16} B/key ({key_b} in, 16 logits out), both parts")}}

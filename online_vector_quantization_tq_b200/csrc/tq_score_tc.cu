@@ -316,7 +316,10 @@ __device__ __forceinline__ void expand_codes(const uint32_t *cw, const uint32_t 
 // Hand-offs are mbarriers only.  Every wait is bounded and gives up as soon
 // as another role has failed, after which all roles leave their loops,
 // in-flight copies and MMAs are waited for (bounded) and TMEM is freed.
-constexpr int kStages = 4;
+// 12 stages of 8 KB (d = 128, b = 4) keep about 100 KB of key rows in flight
+// per SM: enough to cover HBM latency at full bandwidth (4 stages capped the
+// scorer near 3 TB/s)
+constexpr int kStages = 12;
 constexpr int kExpGroups = 1;  // expander groups (four warps each) taking tiles in turn
 constexpr int kExpWarps = 4 * kExpGroups, kEpiWarps = 8;
 constexpr int kMmaWarp = kExpWarps + kEpiWarps;  // and kMmaWarp + 1: the two MMA issuers
@@ -794,7 +797,8 @@ tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int6
   const bool bulk = ng == 4 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
                     (q->m == 0 || reinterpret_cast<uintptr_t>(signs) % 16 == 0);
   if (reinterpret_cast<uintptr_t>(qop) % 16 != 0) return TQ_ERR_ALIGNMENT;
-  const size_t smem = 1024 + (bulk ? kStages * stage_bytes : 0) + 2 * (size_t)N * kScoreKBytes + 8 * 48 + 16;
+  const size_t smem = 1024 + (bulk ? kStages * stage_bytes : 0) + 2 * (size_t)N * kScoreKBytes +
+                      8 * (2 * kStages + 26) + 16;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
