@@ -44,6 +44,7 @@ struct ScoreTCParams {
   float *out;
   int64_t ldo;
   int accumulate;
+  int nstages;  // key-row stages in the ring (bulk copies)
   int *err;
 };
 
@@ -311,14 +312,15 @@ __device__ __forceinline__ void expand_codes(const uint32_t *cw, const uint32_t 
 //                when only one accumulator fits): an issuing thread spends
 //                tens of cycles per tcgen05 instruction, so two of them keep
 //                the tensor core fed;
-//   warp 14      bulk copies: raw key rows into a ring of kStages buffers, and
+//   warp 14      bulk copies: raw key rows into a ring of p.nstages buffers, and
 //                each group's query operand into a ring of two.
 // Hand-offs are mbarriers only.  Every wait is bounded and gives up as soon
 // as another role has failed, after which all roles leave their loops,
 // in-flight copies and MMAs are waited for (bounded) and TMEM is freed.
-// 12 stages of 8 KB (d = 128, b = 4) keep about 100 KB of key rows in flight
-// per SM: enough to cover HBM latency at full bandwidth (4 stages capped the
-// scorer near 3 TB/s)
+// Up to 12 stages of 8 KB (d = 128, b = 4) keep about 100 KB of key rows in
+// flight per SM: enough to cover HBM latency at full bandwidth (4 stages
+// capped the scorer near 3 TB/s).  Fewer when many queries per group leave
+// less shared memory (p.nstages, at least 2).
 constexpr int kStages = 12;
 constexpr int kExpGroups = 1;  // expander groups (four warps each) taking tiles in turn
 constexpr int kExpWarps = 4 * kExpGroups, kEpiWarps = 8;
@@ -377,7 +379,7 @@ struct ScoreSmem {
   static constexpr int kCodeBytes = 128 * kCW * 4;  // per stage
   static constexpr int kSignBytes = 128 * NG * 4;
   static constexpr int kStageBytes = kCodeBytes + kSignBytes;
-  static constexpr int kOffB = kStages * kStageBytes;  // multiple of 1024
+  // the query operands follow the p.nstages stages (stage bytes are a multiple of 1024)
   enum Bar { kFull = 0, kEmpty = kStages, kAFull = 2 * kStages, kAEmpty = kAFull + 4, kAccFull = kAEmpty + 4,
              kAccEmpty = kAccFull + 4, kBFull = kAccEmpty + 4, kBEmpty = kBFull + 2, kMmaDone = kBEmpty + 2,
              kNumBars = kMmaDone + 2 };
@@ -391,7 +393,8 @@ k_score_tc(const ScoreTCParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sStage = smem;
-  uint8_t *sB = smem + (BULK ? SM::kOffB : 0);
+  uint8_t *sB = smem + (BULK ? p.nstages * SM::kStageBytes : 0);
+  const int NS = p.nstages;
   const uint32_t b_bytes = (uint32_t)p.N * kScoreKBytes;  // one query operand
   uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 2 * b_bytes);
   uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + SM::kNumBars);
@@ -406,7 +409,7 @@ k_score_tc(const ScoreTCParams p) {
   const int64_t g0 = t0 / tpg;  // groups are counted from the CTA's first one
   const int nis = tp.nacc >= 2 ? 2 : 1;  // MMA issuers
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < NS; ++i) {
       sm100::mbar_init(&bars[SM::kFull + i], 1);
       sm100::mbar_init(&bars[SM::kEmpty + i], 4);
     }
@@ -462,8 +465,8 @@ k_score_tc(const ScoreTCParams p) {
 #pragma unroll
       for (int k = 0; k < NG; ++k) sw[k] = 0u;
       if constexpr (BULK) {
-        const int slot = it % kStages;
-        if (!__all_sync(0xffffffffu, wait(SM::kFull + slot, (uint32_t)((it / kStages) & 1), 21))) break;
+        const int slot = it % NS;
+        if (!__all_sync(0xffffffffu, wait(SM::kFull + slot, (uint32_t)((it / NS) & 1), 21))) break;
         const uint8_t *st = sStage + slot * SM::kStageBytes;
         if (valid) {
           const uint4 *crow = reinterpret_cast<const uint4 *>(st + row * CW * 4);
@@ -652,8 +655,8 @@ k_score_tc(const ScoreTCParams p) {
         ++b_loaded;
       }
       if constexpr (BULK) {
-        const int jt = (int)issued, slot = jt % kStages;
-        if (jt >= kStages && !wait(SM::kEmpty + slot, (uint32_t)((jt / kStages - 1) & 1), 28)) break;
+        const int jt = (int)issued, slot = jt % NS;
+        if (jt >= NS && !wait(SM::kEmpty + slot, (uint32_t)((jt / NS - 1) & 1), 28)) break;
         const int64_t kin0 = tw.tin * 128;
         const int64_t key0 = tw.g * p.kpg + p.key_base + kin0;
         const int64_t left = p.nkeys - kin0;
@@ -674,11 +677,11 @@ k_score_tc(const ScoreTCParams p) {
     sm100::mbar_wait(&bars[SM::kMmaDone + (warp - kMmaWarp)], 0u, p.err, 29);
   }
   if (warp == kLoadWarp && lane == 0 && *sAbort) {
-    // copies issued but possibly not consumed: the last kStages key stages
+    // copies issued but possibly not consumed: the last p.nstages key stages
     // and the last two query operands
     if constexpr (BULK) {
-      for (int64_t j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        sm100::mbar_wait(&bars[SM::kFull + j % kStages], (uint32_t)((j / kStages) & 1), p.err, 31);
+      for (int64_t j = issued > NS ? issued - NS : 0; j < issued; ++j)
+        sm100::mbar_wait(&bars[SM::kFull + j % NS], (uint32_t)((j / NS) & 1), p.err, 31);
     }
     for (int j = b_loaded > 2 ? b_loaded - 2 : 0; j < b_loaded; ++j)
       sm100::mbar_wait(&bars[SM::kBFull + (j & 1)], (uint32_t)((j >> 1) & 1), p.err, 32);
@@ -797,8 +800,17 @@ tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int6
   const bool bulk = ng == 4 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
                     (q->m == 0 || reinterpret_cast<uintptr_t>(signs) % 16 == 0);
   if (reinterpret_cast<uintptr_t>(qop) % 16 != 0) return TQ_ERR_ALIGNMENT;
-  const size_t smem = 1024 + (bulk ? kStages * stage_bytes : 0) + 2 * (size_t)N * kScoreKBytes +
-                      8 * (2 * kStages + 26) + 16;
+  int max_smem = 0;
+  {
+    int dv = 0;
+    cudaGetDevice(&dv);
+    cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dv);
+  }
+  const size_t fixed = 1024 + 2 * (size_t)N * kScoreKBytes + 8 * (2 * kStages + 26) + 16;
+  int nstages = kStages;
+  while (bulk && nstages > 2 && fixed + nstages * stage_bytes > (size_t)max_smem) --nstages;
+  prm.nstages = nstages;
+  const size_t smem = fixed + (bulk ? nstages * stage_bytes : 0);
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
