@@ -65,6 +65,27 @@ struct DenseGemmParams {
 };
 
 // Split v (|v| 2^e < 2^30) into its four limbs (a, b, c, d).
+// 2^e as a product of two floats (each a power of two inside the normal
+// range for |e| <= 252): v * s.x * s.y is v 2^e exactly, as ldexpf gives it,
+// whenever the result is a normal number.
+__device__ __forceinline__ float2 pow2_pair(int e) {
+  const int e1 = e / 2, e2 = e - e1;
+  return make_float2(__uint_as_float((uint32_t)(127 + e1) << 23), __uint_as_float((uint32_t)(127 + e2) << 23));
+}
+
+// Four signed bytes of round(v 2^e), |v 2^e| < 2^30: 2^24 a + 2^16 b + 2^8 c + d.
+__device__ __forceinline__ uint32_t limb_bytes(float v, float2 s) {
+  int t = __float2int_rn(v * s.x * s.y);
+  uint32_t out = 0u;
+#pragma unroll
+  for (int k = 3; k >= 1; --k) {
+    const int lo = ((t + 128) & 255) - 128;
+    out |= (uint32_t)(uint8_t)lo << (8 * k);
+    t = (t - lo) >> 8;
+  }
+  return out | (uint32_t)(uint8_t)t;  // byte k = limb plane k (plane 0: the top limb)
+}
+
 __device__ __forceinline__ void limbs_of(float v, int e, int8_t (&l)[4]) {
   int t = __float2int_rn(ldexpf(v, e));
 #pragma unroll
@@ -298,11 +319,26 @@ __global__ void k_dense_split(RowSource src, int64_t row0, int64_t rows, int64_t
   frexpf(big, &E);  // big < 2^E
   const int e = big > 0.f ? 30 - E : 0;
   const int64_t plane = plane_rows * d;
-  for (int j = lane; j < d; j += 32) {
-    int8_t l[4];
-    limbs_of(src.at(row0 + row, j), e, l);
+  if (!src.chan && !src.bf16 && d % 128 == 0) {
+    // four consecutive values per lane: one 16-byte load, one 4-byte store per limb plane
+    const float2 sc = pow2_pair(e);
+    const float *xr = static_cast<const float *>(src.x) + (row0 + row) * src.ldx;
+    for (int j = 4 * lane; j < d; j += 128) {
+      const float4 v = *reinterpret_cast<const float4 *>(xr + j);
+      const uint32_t b0 = limb_bytes(v.x, sc), b1 = limb_bytes(v.y, sc), b2 = limb_bytes(v.z, sc),
+                     b3 = limb_bytes(v.w, sc);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) xl[k * plane + row * d + j] = l[k];
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<uint32_t *>(xl + k * plane + row * d + j) =
+            __byte_perm(__byte_perm(b0, b1, 0x40 + 0x11 * k), __byte_perm(b2, b3, 0x40 + 0x11 * k), 0x5410);
+    }
+  } else {
+    for (int j = lane; j < d; j += 32) {
+      int8_t l[4];
+      limbs_of(src.at(row0 + row, j), e, l);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) xl[k * plane + row * d + j] = l[k];
+    }
   }
   if (lane == 0) {
     // the epilogue's integer sum counts units of 2^24
@@ -324,6 +360,19 @@ __global__ void k_dense_rlimbs(const float *r, const unsigned *rmax, int d, int6
   frexpf(big, &E);
   const int e = big > 0.f ? 30 - E : 0;
   const int64_t plane = plane_rows * d;
+  if (d % 128 == 0) {
+    const float2 sc = pow2_pair(e);
+    for (int j = 4 * lane; j < d; j += 128) {
+      const float4 v = *reinterpret_cast<const float4 *>(r + row * d + j);
+      const uint32_t b0 = limb_bytes(v.x, sc), b1 = limb_bytes(v.y, sc), b2 = limb_bytes(v.z, sc),
+                     b3 = limb_bytes(v.w, sc);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<uint32_t *>(rl + k * plane + row * d + j) =
+            __byte_perm(__byte_perm(b0, b1, 0x40 + 0x11 * k), __byte_perm(b2, b3, 0x40 + 0x11 * k), 0x5410);
+    }
+    return;
+  }
   for (int j = lane; j < d; j += 32) {
     int8_t l[4];
     limbs_of(r[row * d + j], e, l);

@@ -322,6 +322,16 @@ __global__ void k_dscore_queries(const float *ytil, const float *p, int d, int m
 template <int W>
 __global__ void k_dscore_keys(KernelTables kt, int64_t cnt, const uint32_t *codes, const uint32_t *signs,
                               const float2 *norms, __half *kop) {
+  // the centroids' two fp16 pieces, c = hi + lo, per code value
+  __shared__ uint16_t tab[2][kMaxLevels];
+  if (threadIdx.x < kMaxLevels) {
+    const float c = kt.centroids[threadIdx.x];
+    const __half hi = __float2half_rn(c);
+    const __half lo = __float2half_rn(c - __half2float(hi));
+    tab[0][threadIdx.x] = *reinterpret_cast<const uint16_t *>(&hi);
+    tab[1][threadIdx.x] = *reinterpret_cast<const uint16_t *>(&lo);
+  }
+  __syncthreads();
   const int ng = kt.d / 32, nsg = kt.m / 32, K = 2 * kt.d + kt.m, per = 2 * ng + nsg;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= cnt * per) return;
@@ -330,22 +340,13 @@ __global__ void k_dscore_keys(KernelTables kt, int64_t cnt, const uint32_t *code
   uint32_t hv[16];
   if (grp < 2 * ng) {
     const int cg = grp < ng ? grp : grp - ng;
-    const bool lo = grp >= ng;
+    const uint16_t *tb = tab[grp >= ng ? 1 : 0];
     uint32_t w[W];
 #pragma unroll
     for (int k = 0; k < W; ++k) w[k] = codes[key * (W * ng) + cg * W + k];
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      float c2[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float c = kt.centroids[unpack_code<W>(w, i + h)];
-        const float chi = __half2float(__float2half_rn(c));
-        c2[h] = lo ? c - chi : chi;
-      }
-      const __half2 h = __floats2half2_rn(c2[0], c2[1]);
-      hv[i / 2] = *reinterpret_cast<const uint32_t *>(&h);
-    }
+    for (int i = 0; i < 32; i += 2)
+      hv[i / 2] = (uint32_t)tb[unpack_code<W>(w, i)] | ((uint32_t)tb[unpack_code<W>(w, i + 1)] << 16);
   } else {
     const uint32_t sw = signs[key * nsg + (grp - 2 * ng)];
     const float g = norms[key].y;
@@ -461,13 +462,21 @@ tq_status dense_score(const tq_quantizer *q, const float *ytil, const float *p, 
   return TQ_OK;
 }
 
+// Keys per chunk of the top-k GEMM: a whole number of key tiles for each of
+// the P CTAs that share a query tile (at most kKeyChunk), so that they finish
+// together.
+static int64_t topk_chunk(int64_t P) {
+  const int64_t per = P * kSBN;
+  return per >= kKeyChunk ? kKeyChunk : (kKeyChunk / per) * per;
+}
+
 size_t dense_topk_ws_bytes(const tq_quantizer *q, int64_t nq, int64_t n) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t ntq = (nq + kSBM - 1) / kSBM;
   const int64_t P = std::max<int64_t>(1, sms / ntq);
-  const int64_t nchunks = (n + kKeyChunk - 1) / kKeyChunk;
+  const int64_t nchunks = (n + topk_chunk(P) - 1) / topk_chunk(P);
   const size_t slots = (size_t)nchunks * P * kTopSlots;
   return up(dense_score_ws_bytes(q, nq)) + up((size_t)nq * slots * 4) + up((size_t)nq * slots * 8);
 }
@@ -494,7 +503,8 @@ tq_status dense_topk(const tq_quantizer *q, const float *ytil, const float *p, i
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const int ntq = (int)((nq + kSBM - 1) / kSBM);
   const int P = std::max(1, sms / ntq);
-  const int64_t nchunks = (n + kKeyChunk - 1) / kKeyChunk;
+  const int64_t chunk = topk_chunk(P);
+  const int64_t nchunks = (n + chunk - 1) / chunk;
   const int64_t slots = nchunks * P * kTopSlots;
   float *part_s = reinterpret_cast<float *>(base + up(L.total));
   int64_t *part_i = reinterpret_cast<int64_t *>(base + up(L.total) + up((size_t)nq * slots * 4));
@@ -512,8 +522,8 @@ tq_status dense_topk(const tq_quantizer *q, const float *ytil, const float *p, i
   auto sw = static_cast<const uint32_t *>(signs);
   auto nr = reinterpret_cast<const float2 *>(norms);
   for (int64_t ci = 0; ci < nchunks; ++ci) {
-    const int64_t key0 = ci * kKeyChunk;
-    const int64_t cnt = std::min(kKeyChunk, n - key0);
+    const int64_t key0 = ci * chunk;
+    const int64_t cnt = std::min(chunk, n - key0);
     const int64_t threads = cnt * (2 * ng + nsg);
     const unsigned blocks = (unsigned)((threads + 255) / 256);
     switch (q->w) {

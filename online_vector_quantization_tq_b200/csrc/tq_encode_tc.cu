@@ -773,13 +773,6 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   float prev_norm = 0.f;
   int64_t prev_row = -1;
   const float2 base2 = make_float2(8388608.0f + (float)HALF, 8388608.0f + (float)HALF);
-  // this thread's 32 columns of the next tile's U, loaded with its norm parts
-  // at the end of the previous iteration (prologue: tile 0)
-  uint32_t acc[32];
-  if (compute && nloc > 0 && !failed) {
-    sm100::tmem_ld32(tmem + lane + kColU0 + 32 * pc, acc);
-    sm100::tmem_wait_ld();
-  }
   int it = 0;
   for (; it < nloc && !failed; ++it) {  // `failed` is CTA-uniform
     const int t = first + it * stride;
@@ -793,6 +786,9 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       const float nrm = nacc * p.rho;
       const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;  // zero rows: u = -0 -> lower middle code
       const float2 sv2 = make_float2(s_v, s_v);
+      uint32_t acc[32];
+      sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
+      sm100::tmem_wait_ld();
       RawPack<W> pk;
       uint32_t hi[16], lo[16];
       float2 g2 = make_float2(0.f, 0.f);
@@ -862,20 +858,12 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         *reinterpret_cast<uint4 *>(sAr + (P + pc) * (kRows * 64) + sm100::sw64_offset(row, k)) =
             make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
       }
-      // ---- (d) the next tile's U (kept for (a)) and norm parts, gamma parts of this one
+      // ---- (d) norm parts of the next tile, gamma parts of this one
       if (it + 1 < nloc) {
         ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 15) && ok;
         ph_rot ^= 1u;
         sm100::tc_fence_after();
-        sm100::tmem_ld32(tmem + lane + (ucol ^ 128u) + 32 * pc, acc);
-        sm100::tmem_wait_ld();
-        float2 ss = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 v = make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1]));
-          ss = __ffma2_rn(v, v, ss);
-        }
-        sm100::tmem_st1(tmem + lane + norm_col(par ^ 1) + pc, __float_as_uint(ss.x + ss.y));
+        row_partial(ucol ^ 128u, norm_col(par ^ 1));
       }
       sm100::tmem_st1(tmem + lane + gam_col(par) + pc, __float_as_uint(g2.x + g2.y));
       sm100::tmem_wait_st();

@@ -378,7 +378,7 @@ struct ScoreSmem {
   static constexpr int kCW = W * NG;                // code words per key
   static constexpr int kCodeBytes = 128 * kCW * 4;  // per stage
   static constexpr int kSignBytes = 128 * NG * 4;
-  static constexpr int kStageBytes = kCodeBytes + kSignBytes;
+  static constexpr int kStageBytes = (kCodeBytes + kSignBytes + 1023) / 1024 * 1024;  // 1024-aligned stages
   // the query operands follow the p.nstages stages (stage bytes are a multiple of 1024)
   enum Bar { kFull = 0, kEmpty = kStages, kAFull = 2 * kStages, kAEmpty = kAFull + 4, kAccFull = kAEmpty + 4,
              kAccEmpty = kAccFull + 4, kBFull = kAccEmpty + 4, kBEmpty = kBFull + 2, kMmaDone = kBEmpty + 2,
@@ -469,21 +469,25 @@ k_score_tc(const ScoreTCParams p) {
         if (!__all_sync(0xffffffffu, wait(SM::kFull + slot, (uint32_t)((it / NS) & 1), 21))) break;
         const uint8_t *st = sStage + slot * SM::kStageBytes;
         if (valid) {
-          const uint4 *crow = reinterpret_cast<const uint4 *>(st + row * CW * 4);
+          if constexpr (CW % 4 == 0) {
+            const uint4 *crow = reinterpret_cast<const uint4 *>(st + row * CW * 4);
 #pragma unroll
-          for (int k = 0; k < CW / 4; ++k) {
-            const uint4 v = crow[k];
-            cw[4 * k] = v.x;
-            cw[4 * k + 1] = v.y;
-            cw[4 * k + 2] = v.z;
-            cw[4 * k + 3] = v.w;
+            for (int k = 0; k < CW / 4; ++k) {
+              const uint4 v = crow[k];
+              cw[4 * k] = v.x;
+              cw[4 * k + 1] = v.y;
+              cw[4 * k + 2] = v.z;
+              cw[4 * k + 3] = v.w;
+            }
+          } else {
+            const uint32_t *crow = reinterpret_cast<const uint32_t *>(st + row * CW * 4);
+#pragma unroll
+            for (int k = 0; k < CW; ++k) cw[k] = crow[k];
           }
           if (p.m > 0) {
-            const uint4 sv = *reinterpret_cast<const uint4 *>(st + SM::kCodeBytes + row * NG * 4);
-            sw[0] = sv.x;
-            sw[1] = sv.y;
-            sw[2] = sv.z;
-            sw[3] = sv.w;
+            const uint32_t *srow = reinterpret_cast<const uint32_t *>(st + SM::kCodeBytes + row * NG * 4);
+#pragma unroll
+            for (int k = 0; k < NG; ++k) sw[k] = srow[k];
           }
         }
         __syncwarp();
@@ -794,10 +798,13 @@ tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int6
   prm.accumulate = accumulate;
   prm.err = q->d_err;
   const int ng = q->d / 32, cwords = q->w * ng;
-  const size_t stage_bytes = (size_t)128 * (cwords + ng) * 4;
+  const size_t stage_bytes = ((size_t)128 * (cwords + ng) * 4 + 1023) / 1024 * 1024;
   // bulk copies need 16-byte aligned starts and sizes: with d = 128 a key's
-  // code and sign rows are multiples of 16 bytes, so any tile qualifies
-  const bool bulk = ng == 4 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
+  // code and sign rows are multiples of 16 bytes, so any tile qualifies;
+  // otherwise every tile's first key and every tile's length must be a
+  // multiple of 4 keys
+  const bool rows4 = key_base % 4 == 0 && kpg % 4 == 0 && nkeys % 4 == 0;
+  const bool bulk = (ng == 4 || rows4) && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
                     (q->m == 0 || reinterpret_cast<uintptr_t>(signs) % 16 == 0);
   if (reinterpret_cast<uintptr_t>(qop) % 16 != 0) return TQ_ERR_ALIGNMENT;
   int max_smem = 0;
@@ -818,7 +825,7 @@ tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int6
   if (grid <= 0) return TQ_OK;
 #define TQ_SC(WW, NGG)                                                                                   \
   {                                                                                                      \
-    auto kern = bulk ? k_score_tc<WW, NGG, (NGG == 4)> : k_score_tc<WW, NGG, false>;                     \
+    auto kern = bulk ? k_score_tc<WW, NGG, true> : k_score_tc<WW, NGG, false>;                           \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
       return TQ_ERR_CUDA;                                                                                \
     kern<<<(unsigned)grid, kScoreThreads, smem, st>>>(prm);                                                        \
