@@ -737,8 +737,9 @@ def run_config(name, args, torch, tq, dev, stream, peak):
         tabs = quantizer_tables_t(torch, q, dev)
         rows = torch.arange(0, n, 16, device=dev)
         e = encs[0]
-        sc = tq.tq_score(q, y[:4], 1, 4, tq.binding.Encoded(e.codes[:kpg:4], e.signs[:kpg:4], e.norms[:kpg:4]),
-                         kpg // 4)
+        sc = tq.tq_score(q, y[:4], 1, 4, tq.binding.Encoded(e.codes[:kpg:4].contiguous(),
+                                                              e.signs[:kpg:4].contiguous(),
+                                                              e.norms[:kpg:4].contiguous()), kpg // 4)
         rec["quality"] = {"encode": encode_quality(torch, q, tabs, x[rows], e.codes[rows], e.signs[rows]),
                           "score": score_quality(torch, q, tabs, y[:4], e.codes[:kpg:4], e.signs[:kpg:4],
                                                  e.norms[:kpg:4], sc),

@@ -123,6 +123,16 @@ class Encoded:
     signs: torch.Tensor   # uint8 [n, sign_bytes]
     norms: torch.Tensor   # float32 [n, 2]: ||x||, gamma
 
+    def check(self):
+        """The library reads and writes whole packed rows back to back: every
+        array must be row-contiguous (a strided view would be read as if it
+        were not)."""
+        for name in ("codes", "signs", "norms"):
+            t = getattr(self, name)
+            if t.numel() and not t.is_contiguous():
+                raise ValueError(f"Encoded.{name} must be contiguous (got strides {t.stride()})")
+        return self
+
 
 class Quantizer:
     """Owned tq_quantizer handle."""
@@ -211,6 +221,7 @@ def tq_encode(q: Quantizer, x: torch.Tensor, out: Encoded | None = None, chan: t
     n = x.shape[0]
     if out is None:
         out = q.empty_encoded(n, x.device)
+    out.check()
     if chan is not None and chan.dtype != torch.int32:
         raise TypeError("chan must be int32")
     L = lib()
@@ -244,6 +255,7 @@ def score_workspace(q: Quantizer, nq: int, device="cuda") -> torch.Tensor:
 def tq_score(q: Quantizer, y: torch.Tensor, groups: int, G: int, enc: Encoded, keys_per_group: int,
              out: torch.Tensor | None = None, accumulate: bool = False, ychan: torch.Tensor | None = None,
              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    enc.check()
     if out is None:
         out = torch.empty((groups * G, keys_per_group), dtype=torch.float32, device=y.device)
     if workspace is None:
@@ -262,6 +274,7 @@ def tq_topk(q: Quantizer, y: torch.Tensor, enc: Encoded, k: int, n: int | None =
             workspace: torch.Tensor | None = None, out=None, stream=None):
     """(scores fp32 [nq, k], key indices int64 [nq, k]); `out` may give both."""
     nq = y.shape[0]
+    enc.check()
     n = enc.codes.shape[0] if n is None else n
     if out is None:
         vals = torch.empty((nq, k), dtype=torch.float32, device=y.device)

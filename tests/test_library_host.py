@@ -129,3 +129,15 @@ def test_mse_mode_tables_match_oracle(tq, d, b):
     for bad in (0, 5):
         with pytest.raises(tq.TQError):
             tq.tq_codebook_mse_host(d, bad, seed=0)
+
+
+def test_encoded_views_must_be_contiguous(tq):
+    """The library reads packed rows back to back, so the binding refuses a
+    strided view of encoded rows (it would be read as if contiguous)."""
+    import torch
+    enc = tq.binding.Encoded(torch.zeros(64, 48, dtype=torch.uint8), torch.zeros(64, 16, dtype=torch.uint8),
+                             torch.zeros(64, 2))
+    enc.check()
+    tq.binding.Encoded(enc.codes[8:], enc.signs[8:], enc.norms[8:]).check()  # a row offset is fine
+    with pytest.raises(ValueError):
+        tq.binding.Encoded(enc.codes[::4], enc.signs[::4], enc.norms[::4]).check()
