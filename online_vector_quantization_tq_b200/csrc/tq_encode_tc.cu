@@ -510,10 +510,12 @@ namespace tq {
 //   u = U / ||U||: the norm comes from the rotated row.
 //
 // 128 * (d/32) threads; thread (row, p) owns columns [32p, 32p+32) of one
-// row.  Per-row partial sums (||U||^2, gamma^2) go through four spare TMEM
-// columns.  The rotation of tile t+1 is issued before the residuals of tile
-// t are computed (U is double-buffered in TMEM), and the sign bits of tile
-// t-1 are read while the QJL projection of tile t is being prepared.
+// row.  Per-row partial sums (||U||^2, gamma^2) go through shared memory.
+// The QJL operand [r_hi | r_lo] is written to TMEM and read from there by
+// the MMA (only S comes from shared memory).  The rotation of tile t+1 is
+// issued before the residuals of tile t are computed (U is double-buffered
+// in TMEM), and the sign bits of tile t-1 are read while the QJL projection
+// of tile t is being prepared.
 // ============================================================================
 namespace {
 
@@ -578,11 +580,11 @@ __device__ __forceinline__ float2 ffma2_rm(float2 a, float2 b, float2 c) {
 template <int D>
 struct Enc2Smem {
   static constexpr int kXBytes = kRows * D * 2;
-  static constexpr int kOffX = 0;                       // 2 x tiles (TMA, 128-byte swizzle)
-  static constexpr int kOffAr = 2 * kXBytes;            // [r_hi | r_lo] fp16, 64-byte swizzle
-  static constexpr int kOffBr = kOffAr + kRows * 2 * D * 2;  // K_hi, K_lo bf16
+  static constexpr int kOffX = 0;                            // 2 x tiles (TMA, 128-byte swizzle)
+  static constexpr int kOffBr = 2 * kXBytes;                 // K_hi, K_lo bf16
   static constexpr int kOffBs = kOffBr + 2 * D * D * 2;      // S fp16
-  static constexpr int kOffMisc = kOffBs + D * D * 2;
+  static constexpr int kOffPart = kOffBs + D * D * 2;        // per-row partial sums, fp32 [2][2][128][4]
+  static constexpr int kOffMisc = kOffPart + 2 * 2 * kRows * 4 * 4;
   static constexpr int kTotal = kOffMisc + 128 + 1024;
 };
 
@@ -598,14 +600,14 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   constexpr int HALF = L / 2;
   constexpr int NB = D / 64;  // TMA boxes of 64 columns
   constexpr int kCompute = 128 * P;  // compute threads; one more warp issues the copies and MMAs
-  constexpr uint32_t kColU0 = 0, kColZ = 256, kColScr = 384;
+  constexpr uint32_t kColU0 = 0, kColZ = 256, kColA = 384;  // U double buffer, QJL accumulator, QJL A operand
   using SM = Enc2Smem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sX = smem + SM::kOffX;
-  uint8_t *sAr = smem + SM::kOffAr;
   uint8_t *sBr = smem + SM::kOffBr;
   uint8_t *sBs = smem + SM::kOffBs;
+  float *sPart = reinterpret_cast<float *>(smem + SM::kOffPart);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffMisc);  // full[2], rot, qjl, drain
   uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 5);
 
@@ -666,14 +668,18 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       }
     sm100::mma_commit(&bars[2]);
   };
+  // The QJL A operand is in TMEM, two fp16 per column: column group pc
+  // holds r_hi of coordinates [32pc, 32pc+32) in its first 16 columns and
+  // r_lo of the same coordinates in the last 16.  K-step ks = 4pc + h reads
+  // columns [32pc + 8h, +8): coordinates 32pc + 16(h & 1) + [0, 16) of r_hi
+  // (h < 2) or r_lo (h >= 2), against the same 16 columns of S.
   auto issue_qjl = [&]() {
-    const uint32_t ar = sm100::smem_u32(sAr), bs = sm100::smem_u32(sBs);
+    const uint32_t bs = sm100::smem_u32(sBs);
 #pragma unroll
     for (int ks = 0; ks < 2 * D / 16; ++ks) {
-      const int kk = ks % (D / 16);
-      const uint64_t a = sm100::desc_sw64(ar + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+      const int kk = 2 * (ks >> 2) + (ks & 1);
       const uint64_t b = sm100::desc_sw64(bs + (kk >> 1) * (D * 64) + (kk & 1) * 32);
-      sm100::mma_f16(tmem + kColZ, a, b, idesc_qjl, ks != 0);
+      sm100::mma_f16_ts(tmem + kColZ, tmem + kColA + 8 * ks, b, idesc_qjl, ks != 0);
     }
     sm100::mma_commit(&bars[3]);
   };
@@ -683,11 +689,11 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     for (int bx = 0; bx < NB; ++bx)
       sm100::tma_load_2d(sX + buf * SM::kXBytes + bx * (kRows * 128), &xmap, bx * 64, tile * kRows, &bars[buf]);
   };
-  // Per-row partial sums live in TMEM columns, double-buffered by tile
-  // parity: ||U||^2 parts at kColScr + 16*par + pc, gamma^2 parts at +8.
-  auto norm_col = [&](int par) { return (uint32_t)(kColScr + 16 * par); };
-  auto gam_col = [&](int par) { return (uint32_t)(kColScr + 16 * par + 8); };
-  auto row_partial = [&](uint32_t ucol, uint32_t scol) {
+  // Per-row partial sums (one per column group) in shared memory,
+  // double-buffered by tile parity: ||U||^2 parts, then gamma^2 parts.
+  auto norm_part = [&](int par) { return sPart + (2 * par) * (kRows * 4) + row * 4; };
+  auto gam_part = [&](int par) { return sPart + (2 * par + 1) * (kRows * 4) + row * 4; };
+  auto row_partial = [&](uint32_t ucol, float *dst) {
     uint32_t u[32];
     sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, u);
     sm100::tmem_wait_ld();
@@ -697,25 +703,27 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       const float2 v = make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1]));
       ss = __ffma2_rn(v, v, ss);
     }
-    sm100::tmem_st1(tmem + lane + scol + pc, __float_as_uint(ss.x + ss.y));
+    dst[pc] = ss.x + ss.y;
   };
-  auto sum_parts = [&](uint32_t scol) {
-    uint32_t parts[4];
-    sm100::tmem_ld4(tmem + lane + scol, parts);
-    sm100::tmem_wait_ld();
+  auto sum_parts = [&](const float *src) {
+    const float4 q4 = *reinterpret_cast<const float4 *>(src);
+    const float parts[4] = {q4.x, q4.y, q4.z, q4.w};
     float v = 0.f;
 #pragma unroll
-    for (int k = 0; k < P; ++k) v += __uint_as_float(parts[k]);
+    for (int k = 0; k < P; ++k) v += parts[k];
     return v;
   };
   auto sign_word = [&]() {
     uint32_t z[32];
     sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
     sm100::tmem_wait_ld();
-    uint32_t wbits = 0u;
+    // four independent chains of eight sign bits
+    uint32_t w8[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
-    return ~wbits;
+    for (int j = 7; j >= 0; --j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w8[c] = __funnelshift_l(z[8 * c + j], w8[c], 1);
+    return ~(w8[0] | (w8[1] << 8) | (w8[2] << 16) | (w8[3] << 24));
   };
 
   // the control thread's bookkeeping of loads in flight
@@ -749,8 +757,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 12);
       ph_rot ^= 1u;
       sm100::tc_fence_after();
-      row_partial(kColU0, norm_col(0));
-      sm100::tmem_wait_st();
+      row_partial(kColU0, norm_part(0));
     }
     sm100::tc_fence_before();
     failed = __syncthreads_or(!ok || ifail) != 0;
@@ -782,7 +789,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     bool ok = true;
     if (compute) {
       // ---- (a) this tile's rotated row (its MMA completed before the last barrier)
-      const float nacc = sqrtf(sum_parts(norm_col(par)));
+      const float nacc = sqrtf(sum_parts(norm_part(par)));
       const float nrm = nacc * p.rho;
       const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;  // zero rows: u = -0 -> lower middle code
       const float2 sv2 = make_float2(s_v, s_v);
@@ -833,7 +840,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       if constexpr (!QJL) {
         // TurboQuant-MSE: no sign bits; the norms of the previous tile
         if (it > 0) {
-          const float gam = pc == 0 ? sqrtf(sum_parts(gam_col(par ^ 1))) * (1.0f / kRScale) : 0.f;
+          const float gam = pc == 0 ? sqrtf(sum_parts(gam_part(par ^ 1))) * (1.0f / kRScale) : 0.f;
           if (pc == 0 && prev_row >= 0 && prev_row < p.n) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
         }
       }
@@ -844,30 +851,31 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         sm100::tc_fence_after();
         // TMEM loads are warp-collective: every lane runs them, only stores are guarded
         const uint32_t sw = sign_word();
-        const float gam = pc == 0 ? sqrtf(sum_parts(gam_col(par ^ 1))) * (1.0f / kRScale) : 0.f;
+        const float gam = pc == 0 ? sqrtf(sum_parts(gam_part(par ^ 1))) * (1.0f / kRScale) : 0.f;
         if (prev_row >= 0 && prev_row < p.n) {
           p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
           if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
         }
       }
-      // ---- (c) residual operand (the previous tile's projection has read it)
+      // ---- (c) residual operand into TMEM (the previous tile's projection has read it)
+      if constexpr (QJL) {
+        uint32_t a32[32];
 #pragma unroll
-      for (int k = 0; k < (QJL ? 4 : 0); ++k) {
-        *reinterpret_cast<uint4 *>(sAr + pc * (kRows * 64) + sm100::sw64_offset(row, k)) =
-            make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
-        *reinterpret_cast<uint4 *>(sAr + (P + pc) * (kRows * 64) + sm100::sw64_offset(row, k)) =
-            make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+        for (int k = 0; k < 16; ++k) {
+          a32[k] = hi[k];
+          a32[16 + k] = lo[k];
+        }
+        sm100::tmem_st32(tmem + lane + kColA + 32 * pc, a32);
       }
       // ---- (d) norm parts of the next tile, gamma parts of this one
       if (it + 1 < nloc) {
         ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 15) && ok;
         ph_rot ^= 1u;
         sm100::tc_fence_after();
-        row_partial(ucol ^ 128u, norm_col(par ^ 1));
+        row_partial(ucol ^ 128u, norm_part(par ^ 1));
       }
-      sm100::tmem_st1(tmem + lane + gam_col(par) + pc, __float_as_uint(g2.x + g2.y));
-      sm100::tmem_wait_st();
-      sm100::fence_proxy_async();
+      gam_part(par)[pc] = g2.x + g2.y;
+      if constexpr (QJL) sm100::tmem_wait_st();
       prev_norm = nrm;
       prev_row = grow;
     }
@@ -900,7 +908,7 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tc_fence_after();
     if (ok && compute) {
       const uint32_t sw = QJL ? sign_word() : 0u;
-      const float gam = pc == 0 ? sqrtf(sum_parts(gam_col((it - 1) & 1))) * (1.0f / kRScale) : 0.f;
+      const float gam = pc == 0 ? sqrtf(sum_parts(gam_part((it - 1) & 1))) * (1.0f / kRScale) : 0.f;
       if (prev_row >= 0 && prev_row < p.n) {
         if (QJL) p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
         if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
@@ -941,10 +949,10 @@ struct EncGSmem {
   static constexpr int kAxBytes = kRows * D * 2;             // one gathered A operand (64-byte swizzle)
   static constexpr int kOffX = 0;
   static constexpr int kOffAx = kOffX + kXBytes;             // two of them
-  static constexpr int kOffAr = kOffAx + 2 * kAxBytes;       // [r_hi | r_lo] fp16
-  static constexpr int kOffBr = kOffAr + kRows * 2 * D * 2;  // RP rotation pieces, bf16
+  static constexpr int kOffBr = kOffAx + 2 * kAxBytes;       // RP rotation pieces, bf16
   static constexpr int kOffBs = kOffBr + RP * D * D * 2;     // S fp16
-  static constexpr int kOffMisc = kOffBs + D * D * 2;
+  static constexpr int kOffPart = kOffBs + D * D * 2;        // per-row partial sums, fp32 [2][2][128][4]
+  static constexpr int kOffMisc = kOffPart + 2 * 2 * kRows * 4 * 4;
   static constexpr int kTotal = kOffMisc + 128 + 1024;
 };
 
@@ -958,15 +966,15 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   constexpr int HALF = L / 2;
   constexpr int NB = SRCW / 64;      // TMA boxes of 64 columns
   constexpr int kCompute = 128 * P;  // compute threads; one more warp issues the copies and MMAs
-  constexpr uint32_t kColU0 = 0, kColZ = 256, kColScr = 384;
+  constexpr uint32_t kColU0 = 0, kColZ = 256, kColA = 384;  // U double buffer, QJL accumulator, QJL A operand
   using SM = EncGSmem<D, RP, SRCW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sX = smem + SM::kOffX;
   uint8_t *sAx = smem + SM::kOffAx;
-  uint8_t *sAr = smem + SM::kOffAr;
   uint8_t *sBr = smem + SM::kOffBr;
   uint8_t *sBs = smem + SM::kOffBs;
+  float *sPart = reinterpret_cast<float *>(smem + SM::kOffPart);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffMisc);  // full, rot, qjl, drain
   uint32_t *sTmem = reinterpret_cast<uint32_t *>(bars + 4);
 
@@ -1026,14 +1034,14 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       }
     sm100::mma_commit(&bars[1]);
   };
+  // The QJL A operand in TMEM, laid out as in k_encode_tc2.
   auto issue_qjl = [&]() {
-    const uint32_t ar = sm100::smem_u32(sAr), bs = sm100::smem_u32(sBs);
+    const uint32_t bs = sm100::smem_u32(sBs);
 #pragma unroll
     for (int ks = 0; ks < 2 * D / 16; ++ks) {
-      const int kk = ks % (D / 16);
-      const uint64_t a = sm100::desc_sw64(ar + (ks >> 1) * (kRows * 64) + (ks & 1) * 32);
+      const int kk = 2 * (ks >> 2) + (ks & 1);
       const uint64_t b = sm100::desc_sw64(bs + (kk >> 1) * (D * 64) + (kk & 1) * 32);
-      sm100::mma_f16(tmem + kColZ, a, b, idesc_qjl, ks != 0);
+      sm100::mma_f16_ts(tmem + kColZ, tmem + kColA + 8 * ks, b, idesc_qjl, ks != 0);
     }
     sm100::mma_commit(&bars[2]);
   };
@@ -1059,9 +1067,9 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
           make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
     sm100::fence_proxy_async();
   };
-  auto norm_col = [&](int par) { return (uint32_t)(kColScr + 16 * par); };
-  auto gam_col = [&](int par) { return (uint32_t)(kColScr + 16 * par + 8); };
-  auto row_partial = [&](uint32_t ucol, uint32_t scol) {
+  auto norm_part = [&](int par) { return sPart + (2 * par) * (kRows * 4) + row * 4; };
+  auto gam_part = [&](int par) { return sPart + (2 * par + 1) * (kRows * 4) + row * 4; };
+  auto row_partial = [&](uint32_t ucol, float *dst) {
     uint32_t u[32];
     sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, u);
     sm100::tmem_wait_ld();
@@ -1071,25 +1079,26 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       const float2 v = make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1]));
       ss = __ffma2_rn(v, v, ss);
     }
-    sm100::tmem_st1(tmem + lane + scol + pc, __float_as_uint(ss.x + ss.y));
+    dst[pc] = ss.x + ss.y;
   };
-  auto sum_parts = [&](uint32_t scol) {
-    uint32_t parts[4];
-    sm100::tmem_ld4(tmem + lane + scol, parts);
-    sm100::tmem_wait_ld();
+  auto sum_parts = [&](const float *src) {
+    const float4 q4 = *reinterpret_cast<const float4 *>(src);
+    const float parts[4] = {q4.x, q4.y, q4.z, q4.w};
     float v = 0.f;
 #pragma unroll
-    for (int k = 0; k < P; ++k) v += __uint_as_float(parts[k]);
+    for (int k = 0; k < P; ++k) v += parts[k];
     return v;
   };
   auto sign_word = [&]() {
     uint32_t z[32];
     sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
     sm100::tmem_wait_ld();
-    uint32_t wbits = 0u;
+    uint32_t w8[4] = {0u, 0u, 0u, 0u};  // four independent chains of eight sign bits
 #pragma unroll
-    for (int j = 31; j >= 0; --j) wbits = __funnelshift_l(z[j], wbits, 1);
-    return ~wbits;
+    for (int j = 7; j >= 0; --j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w8[c] = __funnelshift_l(z[8 * c + j], w8[c], 1);
+    return ~(w8[0] | (w8[1] << 8) | (w8[2] << 16) | (w8[3] << 24));
   };
 
   uint32_t ph_full = 0u, ph_rot = 0u, ph_qjl = 0u;  // compute threads' phases
@@ -1143,8 +1152,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         ok = sm100::mbar_wait(&bars[1], ph_rot, p.err, 62);
         ph_rot ^= 1u;
         sm100::tc_fence_after();
-        row_partial(kColU0, norm_col(0));
-        sm100::tmem_wait_st();
+        row_partial(kColU0, norm_part(0));
       }
       sm100::tc_fence_before();
       failed = __syncthreads_or(!ok) != 0;
@@ -1164,7 +1172,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     bool ok = true;
     if (compute) {
       // ---- (a) codes and residual of this tile
-      const float nacc = sqrtf(sum_parts(norm_col(par)));
+      const float nacc = sqrtf(sum_parts(norm_part(par)));
       const float nrm = nacc * p.rho;
       const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;
       const float2 sv2 = make_float2(s_v, s_v);
@@ -1211,19 +1219,21 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         ph_qjl ^= 1u;
         sm100::tc_fence_after();
         const uint32_t sw = sign_word();
-        const float gam = pc == 0 ? sqrtf(sum_parts(gam_col(par ^ 1))) * (1.0f / kRScale) : 0.f;
+        const float gam = pc == 0 ? sqrtf(sum_parts(gam_part(par ^ 1))) * (1.0f / kRScale) : 0.f;
         if (prev_row >= 0 && prev_row < p.n) {
           p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
           if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
         }
       }
-      // ---- (c) residual operand
+      // ---- (c) residual operand into TMEM (the previous tile's projection has read it)
+      {
+        uint32_t a32[32];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        *reinterpret_cast<uint4 *>(sAr + pc * (kRows * 64) + sm100::sw64_offset(row, k)) =
-            make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
-        *reinterpret_cast<uint4 *>(sAr + (P + pc) * (kRows * 64) + sm100::sw64_offset(row, k)) =
-            make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+        for (int k = 0; k < 16; ++k) {
+          a32[k] = hi[k];
+          a32[16 + k] = lo[k];
+        }
+        sm100::tmem_st32(tmem + lane + kColA + 32 * pc, a32);
       }
       // ---- (g) gather tile it+2 into this tile's A operand (its rotation is done)
       if (it + 2 < nloc) ok = wait_and_gather(first + (it + 2) * stride, par) && ok;
@@ -1232,11 +1242,10 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         ok = sm100::mbar_wait(&bars[1], ph_rot, p.err, 64) && ok;
         ph_rot ^= 1u;
         sm100::tc_fence_after();
-        row_partial(ucol ^ 128u, norm_col(par ^ 1));
+        row_partial(ucol ^ 128u, norm_part(par ^ 1));
       }
-      sm100::tmem_st1(tmem + lane + gam_col(par) + pc, __float_as_uint(g2.x + g2.y));
+      gam_part(par)[pc] = g2.x + g2.y;
       sm100::tmem_wait_st();
-      sm100::fence_proxy_async();
       prev_norm = nrm;
       prev_row = grow;
     }
@@ -1263,7 +1272,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tc_fence_after();
     if (ok && compute) {
       const uint32_t sw = sign_word();
-      const float gam = pc == 0 ? sqrtf(sum_parts(gam_col((it - 1) & 1))) * (1.0f / kRScale) : 0.f;
+      const float gam = pc == 0 ? sqrtf(sum_parts(gam_part((it - 1) & 1))) * (1.0f / kRScale) : 0.f;
       if (prev_row >= 0 && prev_row < p.n) {
         p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
         if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
