@@ -713,17 +713,20 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     for (int k = 0; k < P; ++k) v += parts[k];
     return v;
   };
-  auto sign_word = [&]() {
-    uint32_t z[32];
-    sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
-    sm100::tmem_wait_ld();
-    // four independent chains of eight sign bits
+  // bit j set where Z[j] >= 0 (four independent chains of eight sign bits)
+  auto sign_bits = [](const uint32_t (&z)[32]) {
     uint32_t w8[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int j = 7; j >= 0; --j)
 #pragma unroll
       for (int c = 0; c < 4; ++c) w8[c] = __funnelshift_l(z[8 * c + j], w8[c], 1);
     return ~(w8[0] | (w8[1] << 8) | (w8[2] << 16) | (w8[3] << 24));
+  };
+  auto sign_word = [&]() {
+    uint32_t z[32];
+    sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+    sm100::tmem_wait_ld();
+    return sign_bits(z);
   };
 
   // the control thread's bookkeeping of loads in flight
@@ -788,13 +791,14 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     const int64_t grow = (int64_t)t * kRows + row;
     bool ok = true;
     if (compute) {
-      // ---- (a) this tile's rotated row (its MMA completed before the last barrier)
+      // ---- (a) this tile's rotated row (its MMA completed before the last
+      // barrier), loaded while the row's scale is computed
+      uint32_t acc[32];
+      sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
       const float nacc = sqrtf(sum_parts(norm_part(par)));
       const float nrm = nacc * p.rho;
       const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;  // zero rows: u = -0 -> lower middle code
       const float2 sv2 = make_float2(s_v, s_v);
-      uint32_t acc[32];
-      sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
       sm100::tmem_wait_ld();
       RawPack<W> pk;
       uint32_t hi[16], lo[16];
@@ -844,20 +848,14 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
           if (pc == 0 && prev_row >= 0 && prev_row < p.n) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
         }
       }
-      // ---- (b) sign bits and norms of the previous tile
+      // ---- (b) the previous tile's projection is done: its Z is final and
+      // the residual operand is free
       if (QJL && it > 0) {
         ok = sm100::mbar_wait(&bars[3], ph_qjl, p.err, 14);
         ph_qjl ^= 1u;
         sm100::tc_fence_after();
-        // TMEM loads are warp-collective: every lane runs them, only stores are guarded
-        const uint32_t sw = sign_word();
-        const float gam = pc == 0 ? sqrtf(sum_parts(gam_part(par ^ 1))) * (1.0f / kRScale) : 0.f;
-        if (prev_row >= 0 && prev_row < p.n) {
-          p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
-          if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
-        }
       }
-      // ---- (c) residual operand into TMEM (the previous tile's projection has read it)
+      // ---- (c) residual operand into TMEM
       if constexpr (QJL) {
         uint32_t a32[32];
 #pragma unroll
@@ -866,6 +864,19 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
           a32[16 + k] = lo[k];
         }
         sm100::tmem_st32(tmem + lane + kColA + 32 * pc, a32);
+      }
+      // sign bits and norms of the previous tile (TMEM loads are
+      // warp-collective: every lane runs them, only stores are guarded)
+      if (QJL && it > 0) {
+        uint32_t z[32];
+        sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+        const float gam = pc == 0 ? sqrtf(sum_parts(gam_part(par ^ 1))) * (1.0f / kRScale) : 0.f;
+        sm100::tmem_wait_ld();
+        const uint32_t sw = sign_bits(z);
+        if (prev_row >= 0 && prev_row < p.n) {
+          p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
+          if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
+        }
       }
       // ---- (d) norm parts of the next tile, gamma parts of this one
       if (it + 1 < nloc) {
@@ -882,9 +893,9 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tc_fence_before();
     failed = __syncthreads_or(!ok || ifail) != 0;
     if (failed) break;
-    sm100::tc_fence_after();
     // ---- (e) control thread: QJL projection of this tile, then the rotation two tiles ahead
     if (ctl) {
+      sm100::tc_fence_after();
       if constexpr (QJL) issue_qjl();
       if (it + 3 < nloc) {  // tile it+1's rotation is done with its buffer
         issue_tma(par ^ 1, first + (it + 3) * stride);
