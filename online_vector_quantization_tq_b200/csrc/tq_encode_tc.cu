@@ -1100,16 +1100,20 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     for (int k = 0; k < P; ++k) v += parts[k];
     return v;
   };
-  auto sign_word = [&]() {
-    uint32_t z[32];
-    sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
-    sm100::tmem_wait_ld();
-    uint32_t w8[4] = {0u, 0u, 0u, 0u};  // four independent chains of eight sign bits
+  // bit j set where Z[j] >= 0 (four independent chains of eight sign bits)
+  auto sign_bits = [](const uint32_t (&z)[32]) {
+    uint32_t w8[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int j = 7; j >= 0; --j)
 #pragma unroll
       for (int c = 0; c < 4; ++c) w8[c] = __funnelshift_l(z[8 * c + j], w8[c], 1);
     return ~(w8[0] | (w8[1] << 8) | (w8[2] << 16) | (w8[3] << 24));
+  };
+  auto sign_word = [&]() {
+    uint32_t z[32];
+    sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+    sm100::tmem_wait_ld();
+    return sign_bits(z);
   };
 
   uint32_t ph_full = 0u, ph_rot = 0u, ph_qjl = 0u;  // compute threads' phases
@@ -1182,13 +1186,13 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     const int64_t grow = (int64_t)t * kRows + row;
     bool ok = true;
     if (compute) {
-      // ---- (a) codes and residual of this tile
+      // ---- (a) codes and residual of this tile (U loaded while the scale is computed)
+      uint32_t acc[32];
+      sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
       const float nacc = sqrtf(sum_parts(norm_part(par)));
       const float nrm = nacc * p.rho;
       const float s_v = nacc > 0.f ? kRScale / nacc : -0.0f;
       const float2 sv2 = make_float2(s_v, s_v);
-      uint32_t acc[32];
-      sm100::tmem_ld32(tmem + lane + ucol + 32 * pc, acc);
       sm100::tmem_wait_ld();
       RawPack<W> pk;
       uint32_t hi[16], lo[16];
@@ -1224,19 +1228,14 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
 #pragma unroll
         for (int k = 0; k < W; ++k) dst[k] = cw[k];
       }
-      // ---- (b) sign bits and norms of the previous tile
+      // ---- (b) the previous tile's projection is done: its Z is final and
+      // the residual operand is free
       if (it > 0) {
         ok = sm100::mbar_wait(&bars[2], ph_qjl, p.err, 63);
         ph_qjl ^= 1u;
         sm100::tc_fence_after();
-        const uint32_t sw = sign_word();
-        const float gam = pc == 0 ? sqrtf(sum_parts(gam_part(par ^ 1))) * (1.0f / kRScale) : 0.f;
-        if (prev_row >= 0 && prev_row < p.n) {
-          p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
-          if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
-        }
       }
-      // ---- (c) residual operand into TMEM (the previous tile's projection has read it)
+      // ---- (c) residual operand into TMEM
       {
         uint32_t a32[32];
 #pragma unroll
@@ -1245,6 +1244,18 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
           a32[16 + k] = lo[k];
         }
         sm100::tmem_st32(tmem + lane + kColA + 32 * pc, a32);
+      }
+      // sign bits and norms of the previous tile
+      if (it > 0) {
+        uint32_t z[32];
+        sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
+        const float gam = pc == 0 ? sqrtf(sum_parts(gam_part(par ^ 1))) * (1.0f / kRScale) : 0.f;
+        sm100::tmem_wait_ld();
+        const uint32_t sw = sign_bits(z);
+        if (prev_row >= 0 && prev_row < p.n) {
+          p.signs[prev_row * p.out_stride * (D / 32) + pc] = sw;
+          if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
+        }
       }
       // ---- (g) gather tile it+2 into this tile's A operand (its rotation is done)
       if (it + 2 < nloc) ok = wait_and_gather(first + (it + 2) * stride, par) && ok;
@@ -1263,9 +1274,9 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::tc_fence_before();
     failed = __syncthreads_or(!ok || ifail) != 0;
     if (failed) break;
-    sm100::tc_fence_after();
     // ---- (e) control thread: QJL of this tile, the next raw tile, the rotation two tiles ahead
     if (ctl) {
+      sm100::tc_fence_after();
       issue_qjl();
       if (it + 2 < nloc) pend_full = false;  // consumed by the gather above
       if (it + 3 < nloc) {
