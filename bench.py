@@ -414,6 +414,18 @@ def oracle_rate_for(name):
             dt = time.perf_counter() - t0
             return {"value": x.shape[0] / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
                     "sample": f"the whole workload: 4096 keys encoded + 16 queries top-10, {dt:.2f} s"}
+        if name == "kv_otf":
+            t = o.Tables(128, 4, seed=0)
+            n = 32768
+            x = wl.kv_head_keys(0, 131072)[:n]
+            y = wl.kv_queries()[:4]
+            t0 = time.perf_counter()
+            enc = o.encode(x, t)
+            o.score(*o.prepare_query(y, t), enc, t)
+            dt = time.perf_counter() - t0
+            return {"value": n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
+                    "sample": f"{n} keys of KV head 0 encoded + scored by 4 query heads, {dt:.2f} s (the oracle "
+                              "builds S once per quantizer either way)"}
         if name == "kv_mse":
             t = o.Tables(128, 3, seed=0, mode="mse")
             n = 32768
@@ -745,6 +757,45 @@ def run_config(name, args, torch, tq, dev, stream, peak):
                                                  e.norms[:kpg:4], sc),
                           "inner_product_gain_1_minus_dD": 1.0 - 128 * q.coord_mse,
                           "sample": "encode: every 16th key; score: query heads 0-3 x every 4th key of KV head 0"}
+    elif name == "kv_otf":
+        groups, G, kpg = 8, 4, 131072
+        xs, y_np = kv_keys_host()
+        x = torch.from_numpy(xs).to(dev).to(torch.bfloat16)
+        y = torch.from_numpy(y_np).to(dev)
+        q = tq.tq_codebook(128, 4, seed=0)
+        n = x.shape[0]
+        ref = tq.tq_encode(q, x[:65536])  # stored S, for the bit-identity check
+        tq.tq_set_qjl_onthefly(q, True)
+        encs = [q.empty_encoded(n, dev) for _ in range(2)]
+        logits = torch.empty((groups * G, kpg), dtype=torch.float32, device=dev)
+        ws = tq.score_workspace(q, groups * G, dev)
+        it = [0]
+
+        def step():
+            i = it[0]
+            it[0] += 1
+            ph("encode", lambda: tq.tq_encode(q, x, out=encs[i % 2], stream=stream))
+            ph("score", lambda: tq.tq_score(q, y, groups, G, encs[(i + 1) % 2], kpg, out=logits, workspace=ws,
+                                            stream=stream))
+        ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        pm = ph.mean_ms()
+        kb = q.code_bytes + q.sign_bytes + 8
+        e = encs[0]
+        same = bool(torch.equal(e.codes[:65536], ref.codes) and torch.equal(e.signs[:65536], ref.signs)
+                    and torch.equal(e.norms[:65536], ref.norms))
+        rec = {"workload": "kv_otf: the kv workload with the QJL matrix S generated from the seed inside the "
+                           "encode (per CTA, in shared memory) and the query preparation (per thread, its row) "
+                           "instead of read from the stored table",
+               "value": n / (ms * 1e-3), "unit": "keys/s", "ms_per_step": ms, "phases_ms": pm,
+               "encode_vectors_per_s": n / (pm["encode"] * 1e-3), "score_keys_per_s": n / (pm["score"] * 1e-3),
+               "bytes_per_key": kb,
+               "l2": "two code buffers; each step scores the codes encoded one step earlier",
+               "roofline": {"encode": roofline_hbm(n * (256 + kb), pm["encode"], peak, "k_encode_tc2",
+                                                   f"{256 + kb} B/key (256 in, {kb} out)"),
+                            "score": roofline_hbm(n * (kb + 16), pm["score"], peak, "k_score_tc",
+                                                  f"{kb + 16} B/key ({kb} in, 16 logits out)")},
+               "bit_identical_to_stored_S": {"keys": 65536, "codes_signs_norms_equal": same}}
+        tq.tq_set_qjl_onthefly(q, False)
     elif name == "decode":
         groups, kpg, G = 256, 32768, 4
         q = tq.tq_codebook(128, 3, seed=0)
@@ -899,7 +950,7 @@ def run_tq(args, rank, world, local):
                                   "phases_ms": {"encode": line["encode_ms"], "score": line["score_ms"]},
                                   "roofline": {"encode": line["roofline"], "score": line["score_roofline"]},
                                   "quality": quality, "cpu_baseline": line["cpu_baseline"]}}
-                for name in ("tiny", "kv_mixed", "decode", "ann", "kv_mse", "kv_mixed_2p5"):
+                for name in ("tiny", "kv_mixed", "decode", "ann", "kv_mse", "kv_mixed_2p5", "kv_otf"):
                     configs[name] = run_config(name, args, torch, tq, dev, stream, peak)
                     torch.cuda.empty_cache()
                 line["configs"] = configs
@@ -937,7 +988,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", choices=["all", "kv", "tiny", "kv_mixed", "decode", "ann", "kv_mse",
-                                           "kv_mixed_2p5"], default="all")
+                                           "kv_mixed_2p5", "kv_otf"], default="all")
     ap.add_argument("--queries", type=int, default=1024, help="ann workload: number of queries")
     ap.add_argument("--ann-rows", type=int, default=1_000_000,
                     help="ann workload: database vectors (1e6 is the workload; fewer for profiling captures)")

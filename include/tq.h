@@ -150,6 +150,26 @@ tq_status tq_codebook_get(const tq_quantizer *q, double *centroids,
 tq_status tq_tables_get(const tq_quantizer *q, float *rotation,
                         int8_t *diag_signs, uint16_t *qjl);
 
+/* On-the-fly QJL matrix (TurboQuant article 2.3.2: the random projection is
+ * generated from a pseudo-random sequence instead of being stored).
+ * tq_set_qjl_onthefly(q, enable): with enable != 0 the kernels that can
+ * generate S do so from the quantizer seed instead of reading the stored
+ * table: the bf16 Hadamard encode at d = 64 and 128 (each CTA generates S in
+ * shared memory) and the fused Hadamard query preparation of tq_score at
+ * d <= 128 (each thread generates its row of S).  The generator is the one
+ * described under tq_codebook (SplitMix64 stream 3, Box-Muller in double,
+ * one rounding to fp16), so every output is bit-identical to the stored-S
+ * result; other paths keep reading the table, which stays allocated.
+ * The generation costs time (Box-Muller in double precision per entry);
+ * the stored table is 2*m*d bytes and stays in L2, so the default is off.
+ * Not thread-safe with launches that use q.  TQ_ERR_INVALID_ARG for NULL. */
+tq_status tq_set_qjl_onthefly(tq_quantizer *q, int enable);
+/* tq_qjl_matrix: S (m x d fp16 bit patterns, row-major) generated on the
+ * device by that generator into the caller's device buffer s16 (2*m*d
+ * bytes), on `stream`.  TQ_ERR_UNSUPPORTED for host-only or m = 0
+ * quantizers. */
+tq_status tq_qjl_matrix(const tq_quantizer *q, uint16_t *s16, void *stream);
+
 /* ---------------------------------------------------------------- encode
  * tq_encode: quantize n vectors (TurboQuant article 1.2.3, 2.3, 4.2.1).
  *   x: device, row r at x + r*ldx elements of `dtype`; 16-byte aligned, and

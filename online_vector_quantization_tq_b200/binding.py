@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         "tq_destroy": (None, [vp]),
         "tq_info": (i32, [vp, ctypes.POINTER(_Info)]),
         "tq_code_bytes": (sz, [vp]),
+        "tq_set_qjl_onthefly": (i32, [vp, i32]),
+        "tq_qjl_matrix": (i32, [vp, vp, vp]),
         "tq_codebook_get": (i32, [vp, vp, vp, vp]),
         "tq_tables_get": (i32, [vp, vp, vp, vp]),
         "tq_encode": (i32, [vp, vp, i32, i64, i64, vp, i64, vp, vp, vp, i64, vp]),
@@ -287,6 +289,20 @@ def tq_topk(q: Quantizer, y: torch.Tensor, enc: Encoded, k: int, n: int | None =
         q.handle, _ptr(y), nq, _ld(y), _ptr(enc.codes), _ptr(enc.signs), _ptr(enc.norms), n, k,
         _ptr(vals), _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream)))
     return vals, idx
+
+
+def tq_set_qjl_onthefly(q: Quantizer, enable: bool = True) -> None:
+    """Generate the QJL matrix S from the seed inside the kernels that can
+    (see include/tq.h) instead of reading the stored table."""
+    _check("tq_set_qjl_onthefly", lib().tq_set_qjl_onthefly(q.handle, int(bool(enable))))
+
+
+def tq_qjl_matrix(q: Quantizer, device="cuda", stream=None) -> torch.Tensor:
+    """S (m x d fp16 bit patterns as int16, row-major) generated on the
+    device from the quantizer seed."""
+    out = torch.empty((q.m, q.d), dtype=torch.int16, device=device)
+    _check("tq_qjl_matrix", lib().tq_qjl_matrix(q.handle, _ptr(out), _stream(stream)))
+    return out
 
 
 def tq_rerank(y: torch.Tensor, x: torch.Tensor, cand: torch.Tensor, k: int, out=None, stream=None):

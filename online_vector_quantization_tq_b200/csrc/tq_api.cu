@@ -110,6 +110,18 @@ tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_
                       stream);
 }
 
+tq_status tq_set_qjl_onthefly(tq_quantizer *q, int enable) {
+  if (!q) return TQ_ERR_INVALID_ARG;
+  q->kt.qjl_otf = enable ? 1 : 0;
+  return TQ_OK;
+}
+
+tq_status tq_qjl_matrix(const tq_quantizer *q, uint16_t *s16, void *stream) {
+  if (!q || !s16) return TQ_ERR_INVALID_ARG;
+  if (q->device < 0 || q->m == 0) return TQ_ERR_UNSUPPORTED;
+  return tq::qjl_matrix_launch(q->kt.qjl_key, (int64_t)q->m * q->d, s16, static_cast<cudaStream_t>(stream));
+}
+
 size_t tq_code_bytes(const tq_quantizer *q) {
   if (!q) return 0;
   return (size_t)q->w * q->d / 8 + (size_t)q->m / 8 + 8;

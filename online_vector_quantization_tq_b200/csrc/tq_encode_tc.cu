@@ -21,6 +21,7 @@
 
 #include "tq_common.cuh"
 #include "tq_kernels.h"
+#include "tq_rng.cuh"
 #include "tq_sm100.cuh"
 
 namespace tq {
@@ -30,6 +31,8 @@ struct EncTCParams {
   int ntiles;
   const uint16_t *rot16;  // [RP][D][D] fp16 bits, row-major (out, in)
   const uint16_t *s16;    // [D][D] fp16 bits (QJL rows, in)
+  uint64_t s_key;         // S's stream key, for kernels that generate S
+  int s_otf;              // nonzero: generate S instead of reading s16
   float rho;              // R = rho * sum of rotation pieces
   float thr_s[kMaxLevels];   // thresholds * 2^10
   float cen_s[kMaxLevels];   // centroids * 2^10
@@ -632,7 +635,12 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   }
   sm100::stage_kmajor<D>(sBr, p.rot16, D);
   sm100::stage_kmajor<D>(sBr + D * D * 2, p.rot16 + (size_t)D * D, D);
-  if constexpr (QJL) sm100::stage_kmajor<D>(sBs, p.s16, D);
+  if constexpr (QJL) {
+    if (p.s_otf)
+      generate_kmajor_qjl<D>(sBs, p.s_key);  // S from the seed (TurboQuant article 2.3.2)
+    else
+      sm100::stage_kmajor<D>(sBs, p.s16, D);
+  }
   sm100::fence_proxy_async();
   sm100::tc_fence_before();
   __syncthreads();
@@ -1437,6 +1445,8 @@ tq_status tc2_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ld
   prm.n = n;
   prm.rot16 = q->d_rot_bf16;
   prm.s16 = q->d_qjl16;
+  prm.s_key = q->kt.qjl_key;
+  prm.s_otf = q->kt.qjl_otf;
   prm.rho = q->tc_rho;
   for (int i = 0; i < kMaxLevels; ++i) {
     prm.thr_s[i] = q->kt.thresholds[i] * kRScale;

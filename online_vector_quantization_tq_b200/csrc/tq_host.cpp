@@ -608,6 +608,8 @@ static tq_status build_quantizer(int d, int b, int m, uint64_t seed, tq_rotation
   kt.qjl32 = q->d_qjl32;
   kt.qjl32t = q->d_qjl32t;
   kt.rott = q->d_rott;
+  kt.qjl_key = stream_key(seed, kStreamS);
+  kt.qjl_otf = 0;
   *out = q;
   return TQ_OK;
 }

@@ -24,6 +24,8 @@ struct KernelTables {
   const float *qjl32;                 // m x d fp32 values of S (same numbers)
   const float *qjl32t;                // d x m: S transposed (coalesced S y~ over rows)
   const float *rott;                  // d x d: R transposed (d <= 128; coalesced R y over rows)
+  uint64_t qjl_key;                   // SplitMix64 key of S's stream (entries generated from it)
+  int qjl_otf;                        // nonzero: kernels that can generate S do so instead of reading it
 };
 
 }  // namespace tq

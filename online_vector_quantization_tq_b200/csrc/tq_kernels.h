@@ -58,6 +58,8 @@ tq_status dense_topk(const tq_quantizer *q, const float *ytil, const float *p, i
                      void *ws, size_t ws_bytes, cudaStream_t st);
 
 // Exact re-scoring of candidate keys against raw vectors, then top-k.
+// S generated on the device from its stream key: count fp16 entries, row-major
+tq_status qjl_matrix_launch(uint64_t key, int64_t count, uint16_t *s16, cudaStream_t st);
 tq_status rerank_launch(const float *y, int64_t nq, int64_t ldy, const void *x, bool bf16, int64_t n, int64_t ldx,
                         int d, const int64_t *cand, int kc, int k, float *out_s, int64_t *out_i, cudaStream_t st);
 

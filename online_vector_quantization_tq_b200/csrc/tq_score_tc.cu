@@ -23,6 +23,7 @@
 // article 4.2.2: score against the stored codes without dequantizing).
 #include "tq_common.cuh"
 #include "tq_kernels.h"
+#include "tq_rng.cuh"
 #include "tq_sm100.cuh"
 
 namespace tq {
@@ -161,7 +162,18 @@ k_prep_operand(KernelTables kt, RowSource src, int64_t G, int N, int cexp, int8_
   // p_j = sum_k S[j][k] y~_k: thread j reads row j of S with independent
   // 16-byte loads (one L2 round trip), four partial sums over k mod 4
   float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-  if (kt.m > 0) {  // TurboQuant-MSE quantizers have no QJL projection (p = 0)
+  if (kt.m > 0 && kt.qjl_otf) {
+    // row j of S generated from the seed (TurboQuant article 2.3.2): the
+    // same fp16 values, the same summation order
+    const uint64_t base = (uint64_t)j * D;
+#pragma unroll 4
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      acc0 = fmaf(half_bits_to_float(qjl_entry_f16(kt.qjl_key, base + 4 * k4)), v[4 * k4], acc0);
+      acc1 = fmaf(half_bits_to_float(qjl_entry_f16(kt.qjl_key, base + 4 * k4 + 1)), v[4 * k4 + 1], acc1);
+      acc2 = fmaf(half_bits_to_float(qjl_entry_f16(kt.qjl_key, base + 4 * k4 + 2)), v[4 * k4 + 2], acc2);
+      acc3 = fmaf(half_bits_to_float(qjl_entry_f16(kt.qjl_key, base + 4 * k4 + 3)), v[4 * k4 + 3], acc3);
+    }
+  } else if (kt.m > 0) {  // TurboQuant-MSE quantizers have no QJL projection (p = 0)
     const float4 *srow = reinterpret_cast<const float4 *>(kt.qjl32 + (size_t)j * D);
 #pragma unroll
     for (int k4 = 0; k4 < D / 4; ++k4) {

@@ -565,3 +565,48 @@ def test_gathered_bf16_encode(tq, d, b, rot):
     check_scores(s, o.score(*o.prepare_query(y, t), rep.ref, t), rep.ref["norm"], np.linalg.norm(y, axis=1), d,
                  skip)
     assert np.all(s[:, 11] == 0.0)
+
+
+# ------------------------------------------------------------------ on-the-fly S
+
+@pytest.mark.parametrize("d,seed", [(128, 0), (64, 7), (96, 3), (1536, 0)])
+def test_qjl_matrix_generated_on_device(tq, d, seed):
+    """S generated on the device from the seed (TurboQuant article 2.3.2) is
+    the oracle's S bit for bit: SplitMix64 stream 3, Box-Muller in double,
+    one rounding to fp16."""
+    q = tq.tq_codebook(d, 4, seed=seed)
+    s = tq.tq_qjl_matrix(q).cpu().numpy().view(np.uint16)
+    ref = o.qjl_matrix(d, d, seed).astype(np.float16).view(np.uint16)
+    mism = int(np.count_nonzero(s != ref))
+    assert mism == 0, f"{mism} of {s.size} entries differ"
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_qjl_onthefly_bit_identical(tq, d):
+    """With S generated inside the kernels (the bf16 Hadamard encode and the
+    fused query preparation), codes, signs, norms and logits are bit-identical
+    to the stored-S run, and the codes and logits still match the oracle."""
+    rng = np.random.default_rng(d)
+    n = 40000 + 77  # several tiles per CTA and a ragged last tile
+    x = wl.to_bf16_values(rng.standard_normal((n, d)).astype(np.float32))
+    x[5] = 0.0
+    y = wl.to_bf16_values(rng.standard_normal((8, d)).astype(np.float32))
+    q = tq.tq_codebook(d, 4, seed=0)
+    xd = dev(x, torch.bfloat16)
+    enc0 = tq.tq_encode(q, xd)
+    s0 = tq.tq_score(q, dev(y), 2, 4, enc0, n // 2)
+    tq.tq_set_qjl_onthefly(q, True)
+    enc1 = tq.tq_encode(q, xd)
+    s1 = tq.tq_score(q, dev(y), 2, 4, enc1, n // 2)
+    tq.tq_set_qjl_onthefly(q, False)
+    for a, b in ((enc0.codes, enc1.codes), (enc0.signs, enc1.signs), (enc0.norms, enc1.norms), (s0, s1)):
+        assert torch.equal(a, b)
+    t = tables(d, 4)
+    rep = check_encode(*host(enc1), x, t)
+    kpg = n // 2
+    for g in range(2):
+        rows = slice(g * kpg, (g + 1) * kpg)
+        ref = {k: v[rows] for k, v in rep.ref.items()}
+        yg = y[4 * g:4 * g + 4]
+        check_scores(s1[4 * g:4 * g + 4].cpu().numpy(), o.score(*o.prepare_query(yg, t), ref, t), ref["norm"],
+                     np.linalg.norm(yg, axis=1), d, rep.skip_rows[rows])

@@ -104,6 +104,10 @@ def test_device_calls_refuse_host_only_quantizer(tq):
     assert st == 2
     st = L.tq_encode(None, fake, 0, 16, 128, None, 0, fake, fake, fake, 1, None)
     assert st == 1
+    assert L.tq_qjl_matrix(q.handle, fake, None) == 2  # unsupported: no device tables
+    assert L.tq_qjl_matrix(None, fake, None) == 1
+    assert L.tq_set_qjl_onthefly(None, 1) == 1
+    assert L.tq_set_qjl_onthefly(q.handle, 1) == 0 and L.tq_set_qjl_onthefly(q.handle, 0) == 0
 
 
 def test_layout_is_a_bijection():
