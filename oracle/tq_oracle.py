@@ -40,6 +40,12 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
                                           against D_b, the shrinkage factor
                                           1 - d D_b over random rotations,
                                           and its 2/pi limit at b = 1)
+  dequantize ............................ pinned (codebook points are
+                                          reconstructed exactly, distortion
+                                          d D_b over random vectors)
+  attend (attention consumer) ........... pinned (one key, equal logits =
+                                          mean, shift invariance, a dominant
+                                          logit, planted mistakes)
   outlier_channels ...................... pinned (planted outliers, ties)
   boundary_distance ..................... pinned (enumeration over every
                                           threshold, exact-threshold and
@@ -450,6 +456,36 @@ def boundary_distance(u: np.ndarray, t: Tables) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Two-stage retrieval (TurboQuant article 4.2.2)
 # ---------------------------------------------------------------------------
+
+def dequantize(enc: dict, t: Tables) -> np.ndarray:
+    """Reconstruction from the codebook stage: x_hat = ||x|| R^T c[codes].
+
+    The codes select centroids of the rotated, normalised coordinates
+    (article 1.2.2); rotating back and restoring the stored norm (article
+    4.2.1) gives the TurboQuant-MSE estimate of x (article 4.1.2 dequantizes
+    the cache this way before attention).  Row form: c[codes] @ R."""
+    c = t.centroids[enc["codes"]]
+    return enc["norm"][:, None] * (c @ t.R)
+
+
+def attend(logits: np.ndarray, scale: float, v_enc: dict, t_v: Tables) -> np.ndarray:
+    """Attention output of queries over a quantized KV cache: the softmax
+    over keys of scale * logits, weighting the dequantized values.
+
+    Article 4.1.1 quantizes both keys and values of the cache (the size
+    formula counts both) and recommends TurboQuant-MSE for most heads;
+    article 4.1.2 dequantizes before the attention product.  The pages give
+    no further definition of the value path.  Reading: values are encoded
+    by the same quantizer family in TurboQuant-MSE mode, and the output is
+    softmax(scale * logits) @ dequantize(values), in fp64; the logits are
+    the keys' inner-product estimates (``score``).  ``logits`` is nq x n,
+    the result nq x d."""
+    z = scale * np.asarray(logits, dtype=np.float64)
+    z = z - z.max(axis=1, keepdims=True)
+    w = np.exp(z)
+    w = w / w.sum(axis=1, keepdims=True)
+    return w @ dequantize(v_enc, t_v)
+
 
 def rerank(y: np.ndarray, x: np.ndarray, cand: np.ndarray, k: int):
     """Second stage of two-stage retrieval: the candidates a first stage on

@@ -608,3 +608,70 @@ def test_rerank_planted_mistake(monkeypatch):
     monkeypatch.setattr(o, "rerank", lambda y, x, c, k: real(-y, x, c, k))
     with pytest.raises(AssertionError):
         test_rerank_equals_exact_topk_when_candidates_cover_it()
+
+
+# ---------------------------------------------------------------- attention consumer
+
+def test_dequantize_distortion_norms_and_zero_rows():
+    """The reconstruction ||x|| R^T c[codes] has squared error d D_b per unit
+    of ||x||^2 on random vectors of any norm (the Lloyd-Max distortion of the
+    codebook stage), and a zero row reconstructs to zero.  A reconstruction
+    with R in place of R^T, or without the norm, fails."""
+    d, b = 64, 3
+    t = o.Tables(d, b, seed=4, mode="mse")
+    x = _random_unit(20000, d, 5) * np.exp(np.random.default_rng(6).uniform(-3, 3, (20000, 1)))
+    x[7] = 0.0
+    enc = o.encode(x, t)
+    xh = o.dequantize(enc, t)
+    assert np.all(xh[7] == 0.0)
+    keep = np.arange(x.shape[0]) != 7
+    rel = np.sum((x - xh) ** 2, axis=1)[keep] / np.sum(x * x, axis=1)[keep]
+    assert abs(rel.mean() - d * t.coord_mse) < 4 * rel.std() / math.sqrt(rel.size)
+    wrong_r = enc["norm"][:, None] * (t.centroids[enc["codes"]] @ t.R.T)
+    assert np.mean(np.sum((x - wrong_r) ** 2, axis=1)[keep] / np.sum(x * x, axis=1)[keep]) > 0.5
+    no_norm = t.centroids[enc["codes"]] @ t.R
+    assert np.mean(np.sum((x - no_norm) ** 2, axis=1)[keep] / np.sum(x * x, axis=1)[keep]) > 0.5
+
+
+def test_attend_special_cases():
+    """Softmax attention over dequantized values: a single key returns its
+    reconstruction whatever the logit; equal logits return the mean of the
+    reconstructions; adding a constant to a query's logits changes nothing;
+    a logit far above the others returns that key's reconstruction; the
+    scale multiplies the logits."""
+    d, b = 32, 3
+    t = o.Tables(d, b, seed=8, mode="mse")
+    rng = np.random.default_rng(9)
+    v = rng.standard_normal((50, d)) * rng.uniform(0.1, 10.0, (50, 1))
+    enc = o.encode(v, t)
+    vh = o.dequantize(enc, t)
+    one = {k: a[:1] for k, a in enc.items()}
+    assert np.allclose(o.attend(rng.standard_normal((3, 1)) * 50, 0.7, one, t), vh[:1], rtol=1e-13, atol=0)
+    assert np.allclose(o.attend(np.full((2, 50), 3.25), 1.0, enc, t), np.mean(vh, axis=0)[None, :].repeat(2, 0),
+                       rtol=1e-12, atol=1e-14)
+    s = rng.standard_normal((4, 50)) * 3
+    base = o.attend(s, 0.5, enc, t)
+    assert np.allclose(o.attend(s + np.array([[1.0], [-7.0], [30.0], [0.5]]), 0.5, enc, t), base, rtol=1e-12,
+                       atol=1e-13)
+    assert np.allclose(o.attend(2.0 * s, 0.25, enc, t), base, rtol=1e-12, atol=1e-13)
+    dom = s.copy()
+    dom[1, 17] = 2000.0
+    assert np.allclose(o.attend(dom, 1.0, enc, t)[1], vh[17], rtol=1e-12, atol=1e-13)
+
+
+def test_attend_planted_mistakes(monkeypatch):
+    """A softmax taken over the queries instead of the keys, or one that
+    ignores the scale, fails the special cases."""
+    real = o.attend
+
+    def over_queries(logits, scale, v_enc, t_v):
+        z = scale * np.asarray(logits, dtype=np.float64)
+        w = np.exp(z - z.max(axis=0, keepdims=True))
+        return (w / w.sum(axis=0, keepdims=True)) @ o.dequantize(v_enc, t_v)
+
+    monkeypatch.setattr(o, "attend", over_queries)
+    with pytest.raises(AssertionError):
+        test_attend_special_cases()
+    monkeypatch.setattr(o, "attend", lambda lg, sc, e, t: real(lg, 1.0, e, t))
+    with pytest.raises(AssertionError):
+        test_attend_special_cases()
