@@ -414,6 +414,19 @@ def oracle_rate_for(name):
             dt = time.perf_counter() - t0
             return {"value": x.shape[0] / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
                     "sample": f"the whole workload: 4096 keys encoded + 16 queries top-10, {dt:.2f} s"}
+        if name == "decode_attend":
+            t, tv = o.Tables(128, 3, seed=0), o.Tables(128, 3, seed=0, mode="mse")
+            n = 8192
+            x = wl.decode_group_keys(0, 32768)[:n]
+            v = wl.decode_group_values(0, 32768)[:n]
+            y = wl.decode_queries(1)
+            t0 = time.perf_counter()
+            enc, venc = o.encode(x, t), o.encode(v, tv)
+            o.attend(o.score(*o.prepare_query(y, t), enc, t), 1.0 / math.sqrt(128), venc, tv)
+            dt = time.perf_counter() - t0
+            return {"value": n / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
+                    "sample": f"{n} keys and values of cache 0 encoded, scored by its 4 query heads and attended, "
+                              f"{dt:.2f} s"}
         if name == "kv_otf":
             t = o.Tables(128, 4, seed=0)
             n = 32768
@@ -837,6 +850,60 @@ def run_config(name, args, torch, tq, dev, stream, peak):
                           "score": score_quality(torch, q, tabs, y[:4], cache.codes[:kpg], cache.signs[:kpg],
                                                  cache.norms[:kpg], out[:4]),
                           "sample": "encode: the 256 appended keys; score: all logits of cache 0"}
+    elif name == "decode_attend":
+        groups, kpg, G, bv = 256, 32768, 4, 3
+        q = tq.tq_codebook(128, 3, seed=0)
+        qv = tq.tq_codebook_mse(128, bv, seed=0)
+        cache = q.empty_encoded(groups * kpg, dev)
+        vcache = qv.empty_encoded(groups * kpg, dev)
+        with _pool() as ex:
+            for g0 in range(0, groups, 16):
+                keys = list(ex.map(lambda g: wl.decode_group_keys(g, kpg), range(g0, g0 + 16)))
+                vals = list(ex.map(lambda g: wl.decode_group_values(g, kpg), range(g0, g0 + 16)))
+                for g, xg, vg in zip(range(g0, g0 + 16), keys, vals):
+                    part = tq.binding.Encoded(cache.codes[g * kpg:], cache.signs[g * kpg:], cache.norms[g * kpg:])
+                    tq.tq_encode(q, torch.from_numpy(xg).to(dev).to(torch.bfloat16), out=part, stream=stream)
+                    vpart = tq.binding.Encoded(vcache.codes[g * kpg:], vcache.signs[g * kpg:],
+                                               vcache.norms[g * kpg:])
+                    tq.tq_encode(qv, torch.from_numpy(vg).to(dev).to(torch.bfloat16), out=vpart, stream=stream)
+        y = torch.from_numpy(wl.decode_queries(groups)).to(dev)
+        logits = torch.empty((groups * G, kpg), device=dev)
+        att = torch.empty((groups * G, 128), device=dev)
+        ws = tq.score_workspace(q, groups * G, dev)
+        wsa = tq.binding._workspace(tq.lib().tq_attend_workspace_bytes(qv.handle, groups, G, kpg), dev)
+        scale = 1.0 / math.sqrt(128)
+        n = groups * kpg
+
+        def step():
+            ph("score", lambda: tq.tq_score(q, y, groups, G, cache, kpg, out=logits, workspace=ws, stream=stream))
+            ph("attend", lambda: tq.tq_attend(qv, logits, groups, G, vcache, kpg, scale, out=att, workspace=wsa,
+                                              stream=stream))
+        ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        pm = ph.mean_ms()
+        sb = q.code_bytes + q.sign_bytes + 8 + 4 * G
+        ab = 4 * G + qv.code_bytes + 8
+        rec = {"workload": "decode_attend: the decode caches (256 x 32768 keys, d=128, keys b=3 inner-product mode) "
+                           "with values in TurboQuant-MSE b=3; step = all logits of 4 query heads per cache (tq_score) "
+                           "+ softmax(logits / sqrt(d)) times the dequantized values (tq_attend)",
+               "value": n / (ms * 1e-3), "unit": "keys/s", "ms_per_step": ms, "phases_ms": pm,
+               "attend_keys_per_s": n / (pm["attend"] * 1e-3),
+               "l2": "1.9 GB of key and value codes per step, larger than L2",
+               "roofline": {"score": roofline_hbm(n * sb, pm["score"], peak, "k_score_tc",
+                                                  f"{sb} B/key (56 in, 16 logits out)"),
+                            "attend": roofline_hbm(n * ab, pm["attend"], peak, "k_attend_split",
+                                                   f"{ab} B/key (16 logits, {qv.code_bytes} value codes, "
+                                                   "8 value norms; the second read of the logits hits L2)")}}
+        # quality: group 0's outputs against an fp64 evaluation of the same definition
+        R, _, c, _ = quantizer_tables_t(torch, qv, dev)
+        codes0 = unpack_codes_t(torch, vcache.codes[:kpg], 128, qv.w)
+        vhat = vcache.norms[:kpg, 0].double()[:, None] * (c[codes0] @ R)
+        pr = torch.softmax(scale * logits[:G].double(), dim=1)
+        ref = pr @ vhat
+        floor = pr @ vcache.norms[:kpg, 0].double()
+        err = (att[:G].double() - ref).abs() / floor[:, None]
+        rec["quality"] = {"attend": {"max_err_over_sum_p_norm": float(err.max()),
+                                     "bound_2^-10": 2.0 ** -10,
+                                     "sample": "the 4 query heads of cache 0, every output coordinate"}}
     elif name == "ann":
         n, d, nq = args.ann_rows, 1536, args.queries
         nch = (n + wl.ANN_CHUNK - 1) // wl.ANN_CHUNK
@@ -950,7 +1017,7 @@ def run_tq(args, rank, world, local):
                                   "phases_ms": {"encode": line["encode_ms"], "score": line["score_ms"]},
                                   "roofline": {"encode": line["roofline"], "score": line["score_roofline"]},
                                   "quality": quality, "cpu_baseline": line["cpu_baseline"]}}
-                for name in ("tiny", "kv_mixed", "decode", "ann", "kv_mse", "kv_mixed_2p5", "kv_otf"):
+                for name in ("tiny", "kv_mixed", "decode", "ann", "kv_mse", "kv_mixed_2p5", "kv_otf", "decode_attend"):
                     configs[name] = run_config(name, args, torch, tq, dev, stream, peak)
                     torch.cuda.empty_cache()
                 line["configs"] = configs
@@ -988,7 +1055,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", choices=["all", "kv", "tiny", "kv_mixed", "decode", "ann", "kv_mse",
-                                           "kv_mixed_2p5", "kv_otf"], default="all")
+                                           "kv_mixed_2p5", "kv_otf", "decode_attend"], default="all")
     ap.add_argument("--queries", type=int, default=1024, help="ann workload: number of queries")
     ap.add_argument("--ann-rows", type=int, default=1_000_000,
                     help="ann workload: database vectors (1e6 is the workload; fewer for profiling captures)")

@@ -150,6 +150,38 @@ tq_status tq_codebook_get(const tq_quantizer *q, double *centroids,
 tq_status tq_tables_get(const tq_quantizer *q, float *rotation,
                         int8_t *diag_signs, uint16_t *qjl);
 
+/* ---------------------------------------------------------------- attention
+ * tq_attend: attention of queries over a quantized KV cache (TurboQuant
+ * article 4.1.1: the cache's keys and values are both quantized, with
+ * TurboQuant-MSE recommended for most heads; 4.1.2: the values are
+ * dequantized for the attention product, fp16 on the critical path).
+ *   qv: the values' quantizer: TurboQuant-MSE (tq_codebook_mse), Hadamard,
+ *       d = 64 or 128, b in [2, 4].
+ *   logits: device fp32; row g*G + q at logits + (g*G + q)*ldl holds the
+ *       logits of query q of group g against keys key_base .. key_base +
+ *       nkeys - 1 of the group (tq_score's output layout; ldl >= nkeys).
+ *   scale: multiplies the logits before the softmax (1/sqrt(d) for scaled
+ *       dot-product attention); finite.
+ *   vcodes, vnorms: device, tq_encode(qv) of the values; group g's keys are
+ *       rows [g*keys_per_group, (g+1)*keys_per_group), of which keys
+ *       [key_base, key_base + nkeys) are attended (nkeys >= 1).
+ *   out: device fp32, row g*G + q at out + (g*G + q)*ldo (ldo >= d):
+ *       sum_k softmax_k(scale * logits) v^_k with v^_k = ||v_k|| R^T c[codes_k]
+ *       (the TurboQuant-MSE reconstruction of value k), d floats.
+ *   G in [1, 16]; workspace: device, 16-byte aligned, at least
+ *       tq_attend_workspace_bytes(qv, groups, G, nkeys) bytes (it depends on
+ *       the device's SM count: query it on the device that runs the call).
+ * The weights softmax_k ||v_k|| / max ||v|| and the centroids are fp16, the
+ * products are accumulated in fp32 on the tensor cores: each output
+ * coordinate is within about 2^-10 sum_k softmax_k ||v_k|| of the exact
+ * value.  groups == 0 or G == 0: no-op.  Other d, b, rotation or a
+ * non-MSE quantizer: TQ_ERR_UNSUPPORTED. */
+size_t tq_attend_workspace_bytes(const tq_quantizer *qv, int64_t groups, int64_t G, int64_t nkeys);
+tq_status tq_attend(const tq_quantizer *qv, const float *logits, int64_t ldl, int64_t groups,
+                    int64_t G, float scale, const void *vcodes, const float *vnorms,
+                    int64_t keys_per_group, int64_t key_base, int64_t nkeys, float *out,
+                    int64_t ldo, void *workspace, size_t workspace_bytes, void *stream);
+
 /* On-the-fly QJL matrix (TurboQuant article 2.3.2: the random projection is
  * generated from a pseudo-random sequence instead of being stored).
  * tq_set_qjl_onthefly(q, enable): with enable != 0 the kernels that can

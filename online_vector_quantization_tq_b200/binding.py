@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         "tq_info": (i32, [vp, ctypes.POINTER(_Info)]),
         "tq_code_bytes": (sz, [vp]),
         "tq_set_qjl_onthefly": (i32, [vp, i32]),
+        "tq_attend_workspace_bytes": (sz, [vp, i64, i64, i64]),
+        "tq_attend": (i32, [vp, vp, i64, i64, i64, ctypes.c_float, vp, vp, i64, i64, i64, vp, i64, vp, sz, vp]),
         "tq_qjl_matrix": (i32, [vp, vp, vp]),
         "tq_codebook_get": (i32, [vp, vp, vp, vp]),
         "tq_tables_get": (i32, [vp, vp, vp, vp]),
@@ -289,6 +291,25 @@ def tq_topk(q: Quantizer, y: torch.Tensor, enc: Encoded, k: int, n: int | None =
         q.handle, _ptr(y), nq, _ld(y), _ptr(enc.codes), _ptr(enc.signs), _ptr(enc.norms), n, k,
         _ptr(vals), _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream)))
     return vals, idx
+
+
+def tq_attend(qv: Quantizer, logits: torch.Tensor, groups: int, G: int, venc: Encoded, keys_per_group: int,
+              scale: float, key_base: int = 0, nkeys: int | None = None, out: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Attention over a quantized KV cache: softmax(scale * logits) times the
+    TurboQuant-MSE reconstructions of the values (venc, encoded by qv), one
+    row of d floats per query (groups*G rows)."""
+    venc.check()
+    n = keys_per_group - key_base if nkeys is None else nkeys
+    if out is None:
+        out = torch.empty((groups * G, qv.d), dtype=torch.float32, device=logits.device)
+    if workspace is None:
+        workspace = _workspace(lib().tq_attend_workspace_bytes(qv.handle, groups, G, n), logits.device)
+    _check("tq_attend", lib().tq_attend(
+        qv.handle, _ptr(logits), _ld(logits), groups, G, float(scale), _ptr(venc.codes),
+        _ptr(venc.norms), keys_per_group, key_base, n, _ptr(out), _ld(out), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return out
 
 
 def tq_set_qjl_onthefly(q: Quantizer, enable: bool = True) -> None:

@@ -2,6 +2,7 @@
 // preparation, scoring, top-k, outlier-channel choice).  Argument checks
 // happen here, before anything is launched; see include/tq.h for the
 // contract of each call.
+#include <cmath>
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -108,6 +109,32 @@ tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype dtype, int64_
   }
   return tq_encode_ws(q, x, dtype, n, ldx, chan, chan_rows, codes, signs, norms, out_stride, nullptr, 0,
                       stream);
+}
+
+size_t tq_attend_workspace_bytes(const tq_quantizer *qv, int64_t groups, int64_t G, int64_t nkeys) {
+  if (!qv || groups < 0 || G < 0 || nkeys < 0) return 0;
+  if (groups == 0 || G == 0 || nkeys == 0 || qv->device < 0) return 0;
+  DeviceGuard g(qv->device);
+  if (!g.ok) return 0;
+  return tq::attend_ws_bytes(groups, G, qv->d, nkeys);
+}
+
+tq_status tq_attend(const tq_quantizer *qv, const float *logits, int64_t ldl, int64_t groups, int64_t G,
+                    float scale, const void *vcodes, const float *vnorms, int64_t keys_per_group, int64_t key_base,
+                    int64_t nkeys, float *out, int64_t ldo, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!qv || groups < 0 || G < 0 || keys_per_group < 0 || key_base < 0 || nkeys < 0) return TQ_ERR_INVALID_ARG;
+  if (qv->device < 0 || !tq::attend_supported(qv)) return TQ_ERR_UNSUPPORTED;
+  if (groups == 0 || G == 0) return TQ_OK;
+  if (G > 16) return TQ_ERR_UNSUPPORTED;
+  if (nkeys == 0 || key_base + nkeys > keys_per_group || ldl < nkeys || ldo < qv->d) return TQ_ERR_INVALID_ARG;
+  if (!logits || !vcodes || !vnorms || !out || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+  if (!aligned(logits, 4) || !aligned(vcodes, 4) || !aligned(vnorms, 8) || !aligned(out, 4)) return TQ_ERR_ALIGNMENT;
+  if (!workspace || !aligned(workspace, 16)) return TQ_ERR_WORKSPACE;
+  DeviceGuard g(qv->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  if (workspace_bytes < tq::attend_ws_bytes(groups, G, qv->d, nkeys)) return TQ_ERR_WORKSPACE;
+  return tq::attend_launch(qv, logits, ldl, groups, G, scale, vcodes, vnorms, keys_per_group, key_base, nkeys, out,
+                           ldo, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 tq_status tq_set_qjl_onthefly(tq_quantizer *q, int enable) {

@@ -58,6 +58,12 @@ tq_status dense_topk(const tq_quantizer *q, const float *ytil, const float *p, i
                      void *ws, size_t ws_bytes, cudaStream_t st);
 
 // Exact re-scoring of candidate keys against raw vectors, then top-k.
+// attention over a quantized KV cache (values in TurboQuant-MSE)
+bool attend_supported(const tq_quantizer *qv);
+size_t attend_ws_bytes(int64_t groups, int64_t G, int d, int64_t nkeys);
+tq_status attend_launch(const tq_quantizer *qv, const float *logits, int64_t ldl, int64_t groups, int64_t G,
+                        float scale, const void *vcodes, const float *vnorms, int64_t kpg, int64_t key_base,
+                        int64_t nkeys, float *out, int64_t ldo, void *ws, size_t ws_bytes, cudaStream_t st);
 // S generated on the device from its stream key: count fp16 entries, row-major
 tq_status qjl_matrix_launch(uint64_t key, int64_t count, uint16_t *s16, cudaStream_t st);
 tq_status rerank_launch(const float *y, int64_t nq, int64_t ldy, const void *x, bool bf16, int64_t n, int64_t ldx,

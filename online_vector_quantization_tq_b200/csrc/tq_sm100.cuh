@@ -272,6 +272,21 @@ __device__ __forceinline__ uint64_t desc_sw64(uint32_t smem_addr, uint32_t sbo =
 
 // Same for the 128-byte swizzle (the layout TMA writes with
 // CU_TENSOR_MAP_SWIZZLE_128B): 8-row x 128-byte atoms, 1024-byte aligned.
+// Shared-memory descriptor for an MN-major operand with the 128-byte
+// swizzle: atoms of 8 K-rows x 128 bytes (64 fp16 along MN, rows 128 B
+// apart, 16-byte chunks XOR-swizzled by the row as TMA's 128-byte swizzle
+// does), MN blocks of 64 elements `lbo` bytes apart, groups of 8 K-rows
+// `sbo` bytes apart.  Atoms must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;                  // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                  // swizzle mode: 128 B
+  return d;
+}
+
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t smem_addr, uint32_t sbo = 1024) {
   uint64_t d = 0;
   d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
@@ -293,6 +308,18 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
          | (0u << 7) | (0u << 10)       // A, B: f16
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// Instruction descriptor, kind::f16, fp16 A (K-major) and fp16 B (MN-major),
+// fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
+  return idesc_f16_f32(M, N) | (1u << 16);  // B major: MN
+}
+
+// Instruction descriptor, kind::f16, fp16 A (MN-major) and fp16 B (K-major),
+// fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_f16_f32_amn(int M, int N) {
+  return idesc_f16_f32(M, N) | (1u << 15);  // A major: MN
 }
 
 // Instruction descriptor, kind::i8, signed 8-bit A and B (K-major), s32 accumulate.

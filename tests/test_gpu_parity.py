@@ -610,3 +610,69 @@ def test_qjl_onthefly_bit_identical(tq, d):
         yg = y[4 * g:4 * g + 4]
         check_scores(s1[4 * g:4 * g + 4].cpu().numpy(), o.score(*o.prepare_query(yg, t), ref, t), ref["norm"],
                      np.linalg.norm(yg, axis=1), d, rep.skip_rows[rows])
+
+
+# ------------------------------------------------------------------ attention consumer
+
+@pytest.mark.parametrize("d,b,G,nkeys,groups", [(128, 3, 4, 9000, 3), (64, 2, 3, 1001, 2), (128, 4, 8, 130, 5),
+                                                 (128, 3, 16, 700, 1)])
+def test_attend_against_oracle(tq, d, b, G, nkeys, groups):
+    """Attention over a quantized cache: keys in inner-product mode scored
+    by tq_score, values in TurboQuant-MSE mode.  The value codes are checked
+    against the oracle's encode; tq_attend's output against the oracle's
+    softmax over the same logits weighting the reconstructions of the same
+    codes.  A key window that starts inside each group, ragged tiles, value
+    norms over 2.6 decades.  Tolerance per coordinate: 2^-10 sum_k p_k ||v_k||
+    (fp16 weights and centroids: two roundings of 2^-11 each) + 1e-6."""
+    rng = np.random.default_rng(d * 10 + b + G)
+    key_base = 17
+    kpg = key_base + nkeys + 40
+    n = groups * kpg
+    kx = wl.to_bf16_values(rng.standard_normal((n, d)).astype(np.float32))
+    vx = wl.to_bf16_values((rng.standard_normal((n, d)) * rng.uniform(0.05, 20.0, (n, 1))).astype(np.float32))
+    y = wl.to_bf16_values(rng.standard_normal((groups * G, d)).astype(np.float32) * 2.0)
+    qk = tq.tq_codebook(d, 4, seed=0)
+    qv = tq.tq_codebook_mse(d, b, seed=0)
+    kenc = tq.tq_encode(qk, dev(kx, torch.bfloat16))
+    venc = tq.tq_encode(qv, dev(vx, torch.bfloat16))
+    logits = tq.tq_score(qk, dev(y), groups, G, kenc, kpg)
+    scale = 1.0 / math.sqrt(d)
+    out = tq.tq_attend(qv, logits[:, key_base:], groups, G, venc, kpg, scale, key_base=key_base,
+                       nkeys=nkeys).cpu().numpy()
+    tv = tables_mse(d, b)
+    codes, signs, norms = host(venc)
+    check_encode(codes, signs, norms, vx, tv)
+    from tests.layout import unpack_codes
+    vcodes = unpack_codes(codes, d, tv.w)
+    lg = logits.cpu().numpy().astype(np.float64)
+    worst = 0.0
+    for g in range(groups):
+        rows = slice(g * kpg + key_base, g * kpg + key_base + nkeys)
+        ve = {"codes": vcodes[rows], "norm": norms[rows, 0].astype(np.float64)}
+        ls = lg[g * G:(g + 1) * G, key_base:key_base + nkeys]
+        ref = o.attend(ls, scale, ve, tv)
+        z = scale * ls
+        p = np.exp(z - z.max(axis=1, keepdims=True))
+        floor = (p / p.sum(axis=1, keepdims=True)) @ ve["norm"]
+        err = np.abs(out[g * G:(g + 1) * G] - ref)
+        bound = 2.0 ** -10 * floor[:, None] + 1e-6
+        assert np.all(err <= bound), f"group {g}: worst {np.max(err / bound):.3f} of the bound"
+        worst = max(worst, float(np.max(err / floor[:, None])))
+    print(f"attend d={d} b={b} G={G}: worst error {worst:.2e} of sum p ||v||")
+
+
+def test_attend_argument_checks(tq):
+    """Unsupported value quantizers and bad windows are refused before any
+    launch."""
+    qv = tq.tq_codebook_mse(128, 3, seed=0)
+    qk = tq.tq_codebook(128, 4, seed=0)  # inner-product mode: not a value quantizer here
+    venc = tq.tq_encode(qv, torch.zeros((256, 128), dtype=torch.bfloat16, device="cuda"))
+    logits = torch.zeros((4, 256), device="cuda")
+    with pytest.raises(tq.TQError):
+        tq.tq_attend(qk, logits, 1, 4, venc, 256, 0.1)
+    with pytest.raises(tq.TQError):
+        tq.tq_attend(qv, logits, 1, 4, venc, 256, 0.1, key_base=200, nkeys=100)
+    with pytest.raises(tq.TQError):
+        tq.tq_attend(qv, logits, 1, 4, venc, 256, float("nan"))
+    out = tq.tq_attend(qv, logits, 1, 4, venc, 256, 0.1)  # zero values: zero output
+    assert torch.all(out == 0)

@@ -24,6 +24,8 @@ from __future__ import annotations
 
 from dataclasses import dataclass
 
+import math
+
 import numpy as np
 
 CONFIG_INDEX = {"tiny": 0, "kv": 1, "kv_mixed": 2, "decode": 3, "ann": 4}
@@ -121,6 +123,15 @@ def decode_group_keys(group: int, n: int = 32768) -> np.ndarray:
     group = sequence * 8 + head.  Row n-1 is the key the decode step appends."""
     rng = np.random.default_rng([data_seed("decode"), group])
     return to_bf16_values(rng.standard_normal((n, 128), dtype=np.float32))
+
+
+def decode_group_values(group: int, n: int = 32768) -> np.ndarray:
+    """Values of the same cache, bf16-exact float32 [n, 128]: N(0,1) rows
+    times a per-row scale drawn log-uniformly from [1/4, 4]."""
+    rng = np.random.default_rng([data_seed("decode"), group, 1])
+    v = rng.standard_normal((n, 128), dtype=np.float32)
+    v *= np.exp(rng.uniform(-math.log(4.0), math.log(4.0), (n, 1))).astype(np.float32)
+    return to_bf16_values(v)
 
 
 def decode_queries(groups: int = 256) -> np.ndarray:
