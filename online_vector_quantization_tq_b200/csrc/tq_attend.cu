@@ -351,10 +351,12 @@ k_attend_combine(KernelTables kt, int64_t G, int64_t nsplit, const float *part_o
 }
 
 int attend_nsplit(int64_t groups, int64_t nkeys, int sms, int64_t *split_keys) {
-  // about two work items per resident CTA (three per SM), ranges of at least four tiles
+  // At least about two work items per resident CTA (three per SM), ranges of
+  // at least four tiles; and ranges of at most 16 tiles, so that a range's
+  // logits are still in L2 when its second pass reads them again.
   const int64_t want = std::max<int64_t>(1, (6 * (int64_t)sms + groups - 1) / groups);
   const int64_t by_len = std::max<int64_t>(1, (nkeys + 4 * kAttTile - 1) / (4 * kAttTile));
-  const int64_t ns = std::min(want, by_len);
+  const int64_t ns = std::max(std::min(want, by_len), (nkeys + 16 * kAttTile - 1) / (16 * kAttTile));
   const int64_t per = (nkeys + ns - 1) / ns;
   *split_keys = (per + kAttTile - 1) / kAttTile * kAttTile;
   return (int)((nkeys + *split_keys - 1) / *split_keys);
