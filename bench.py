@@ -50,12 +50,16 @@ import numpy as np  # noqa: E402
 METRIC = "keys scored/s and vectors encoded/s (1 B200), as % of HBM roofline"
 CSRC = os.path.join(ROOT, "online_vector_quantization_tq_b200", "csrc")
 
-# DRAM bytes (read + write) per launch counted by ncu for a kernel, with the
-# SHA-256 (first 16 hex digits) of the source file it was built from at the
-# time of the capture.  A figure is reported only while the source is
-# unchanged; otherwise the roofline's traffic is null.
+# DRAM bytes (read + write) per launch counted by ncu for a kernel on one
+# workload ("kernel@workload"), with the SHA-256 (first 16 hex digits) of the
+# source file it was built from at the time of the capture.  A figure is
+# reported only for that workload and while the source is unchanged;
+# otherwise the roofline's traffic is null.
 TRAFFIC = {
-    # kernel: (source file, digest, bytes per launch, workload of the capture)
+    # kernel@workload: (source file, digest, bytes per launch, the capture)
+    "k_encode_tc2@kv": ("tq_encode_tc.cu", "35b4e65c17d1aeec", 326967296, "kv workload, launch 4, ncu --set full"),
+    "k_score_tc@kv": ("tq_score_tc.cu", "f3d48b916b85d13a", 79352832, "kv workload, launch 4, ncu --set full"),
+    "k_attend_split@decode_attend": ("tq_attend.cu", "92d847b55e84b554", 615426816, "decode_attend workload, launch 3, ncu --set full"),
 }
 
 
@@ -64,8 +68,8 @@ def _source_digest(fname: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_for(kernel: str):
-    ent = TRAFFIC.get(kernel)
+def traffic_for(kernel: str, workload=None):
+    ent = TRAFFIC.get(f"{kernel}@{workload}") if workload else None
     if not ent:
         return None, None
     fname, digest, nbytes, where = ent
@@ -213,8 +217,8 @@ def timed_steps(torch, dev, stream, step, steps, warmup, phases=None, clock=None
     return t0.elapsed_time(t1) / steps
 
 
-def roofline_hbm(algo_bytes, ms, peak, kernel, unit_note):
-    traffic, where = traffic_for(kernel)
+def roofline_hbm(algo_bytes, ms, peak, kernel, unit_note, workload=None):
+    traffic, where = traffic_for(kernel, workload)
     achieved = algo_bytes / (ms * 1e-3) / 1e9
     r = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak["hbm_gbs"],
          "peak_kind": peak["kind"], "unit": "GB/s", "frac": achieved / peak["hbm_gbs"],
@@ -225,8 +229,8 @@ def roofline_hbm(algo_bytes, ms, peak, kernel, unit_note):
     return r
 
 
-def roofline_tensor(algo_flops, ms, peak, kernel, unit_note):
-    traffic, where = traffic_for(kernel)
+def roofline_tensor(algo_flops, ms, peak, kernel, unit_note, workload=None):
+    traffic, where = traffic_for(kernel, workload)
     achieved = algo_flops / (ms * 1e-3) / 1e12
     r = {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": peak["bf16_tflops_sustained"],
          "peak_kind": peak["kind"] + " (bf16 dense, sustained)", "unit": "TFLOP/s",
@@ -619,9 +623,11 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
         "encode_ms": enc_ms,
         "score_ms": score_ms,
         "roofline": roofline_hbm(n * enc_bytes_key, enc_ms, peak, "k_encode_tc2",
-                                 f"{enc_bytes_key} B/key (256 in, 48 codes + 16 signs + 8 norms out) x {n} keys"),
+                                 f"{enc_bytes_key} B/key (256 in, 48 codes + 16 signs + 8 norms out) x {n} keys",
+                                 workload="kv"),
         "score_roofline": dict(roofline_hbm(n * score_bytes_key, score_ms, peak, "k_score_tc",
-                                            f"{score_bytes_key} B/key (72 in, 4 logits x 4 B out) x {n} keys"),
+                                            f"{score_bytes_key} B/key (72 in, 4 logits x 4 B out) x {n} keys",
+                                            workload="kv"),
                                note="phase time: the fused query preparation kernel + the scorer"),
         "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "keys/s",
                 "h2d_bytes_per_step": x_pin.numel() * 2 + y_pin.numel() * 4,
@@ -892,7 +898,8 @@ def run_config(name, args, torch, tq, dev, stream, peak):
                                                   f"{sb} B/key (56 in, 16 logits out)"),
                             "attend": roofline_hbm(n * ab, pm["attend"], peak, "k_attend_split",
                                                    f"{ab} B/key (16 logits, {qv.code_bytes} value codes, "
-                                                   "8 value norms; the second read of the logits hits L2)")}}
+                                                   "8 value norms; the second read of the logits hits L2)",
+                                                   workload="decode_attend")}}
         # quality: group 0's outputs against an fp64 evaluation of the same definition
         R, _, c, _ = quantizer_tables_t(torch, qv, dev)
         codes0 = unpack_codes_t(torch, vcache.codes[:kpg], 128, qv.w)

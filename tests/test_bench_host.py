@@ -55,8 +55,10 @@ def test_torch_unpackers_match_the_layout_helper():
 def test_traffic_is_null_once_the_source_changes(monkeypatch):
     b = _bench()
     digest = b._source_digest("tq_api.cu")
-    monkeypatch.setattr(b, "TRAFFIC", {"k": ("tq_api.cu", digest, 123, "small case"),
-                                       "old": ("tq_api.cu", "0" * 16, 456, "small case")})
-    assert b.traffic_for("k") == (123, "small case")
-    assert b.traffic_for("old") == (None, None)
-    assert b.traffic_for("missing") == (None, None)
+    monkeypatch.setattr(b, "TRAFFIC", {"k@w": ("tq_api.cu", digest, 123, "small case"),
+                                       "old@w": ("tq_api.cu", "0" * 16, 456, "small case")})
+    assert b.traffic_for("k", "w") == (123, "small case")
+    assert b.traffic_for("k", "other") == (None, None)  # a capture holds for its own workload only
+    assert b.traffic_for("k") == (None, None)
+    assert b.traffic_for("old", "w") == (None, None)
+    assert b.traffic_for("missing", "w") == (None, None)
