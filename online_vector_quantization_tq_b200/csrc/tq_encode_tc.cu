@@ -791,14 +791,20 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   float prev_norm = 0.f;
   int64_t prev_row = -1;
   const float2 base2 = make_float2(8388608.0f + (float)HALF, 8388608.0f + (float)HALF);
+  // The compute warps and the issuing warp run separate copies of the tile
+  // loop (each keeps only its own code in the instruction stream), meeting
+  // once per tile at one named barrier that also votes on failures; both
+  // copies take the same number of iterations because `failed` comes from
+  // that vote.
+  constexpr int kThreadsAll = kCompute + 32;
   int it = 0;
-  for (; it < nloc && !failed; ++it) {  // `failed` is CTA-uniform
+  if (compute) for (; it < nloc && !failed; ++it) {  // `failed` is CTA-uniform
     const int t = first + it * stride;
     const int par = it & 1;
     const uint32_t ucol = par ? 128u : 0u;
     const int64_t grow = (int64_t)t * kRows + row;
     bool ok = true;
-    if (compute) {
+    {
       // ---- (a) this tile's rotated row (its MMA completed before the last
       // barrier), loaded while the row's scale is computed
       uint32_t acc[32];
@@ -873,8 +879,16 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         }
         sm100::tmem_st32(tmem + lane + kColA + 32 * pc, a32);
       }
-      // sign bits and norms of the previous tile (TMEM loads are
-      // warp-collective: every lane runs them, only stores are guarded)
+      // ---- (d) once the next tile's rotation is done (the tensor core no
+      // longer writes TMEM, so the loads are quick): Z of the previous tile
+      // for its sign bits and norms, then the next tile's U for its norm
+      // parts (TMEM loads are warp-collective: every lane runs them, only
+      // stores are guarded)
+      if (it + 1 < nloc) {
+        ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 15) && ok;
+        ph_rot ^= 1u;
+        sm100::tc_fence_after();
+      }
       if (QJL && it > 0) {
         uint32_t z[32];
         sm100::tmem_ld32(tmem + lane + kColZ + 32 * pc, z);
@@ -886,20 +900,20 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
           if (pc == 0) p.norms[prev_row * p.out_stride] = make_float2(prev_norm, gam);
         }
       }
-      // ---- (d) norm parts of the next tile, gamma parts of this one
-      if (it + 1 < nloc) {
-        ok = sm100::mbar_wait(&bars[2], ph_rot, p.err, 15) && ok;
-        ph_rot ^= 1u;
-        sm100::tc_fence_after();
-        row_partial(ucol ^ 128u, norm_part(par ^ 1));
-      }
+      if (it + 1 < nloc) row_partial(ucol ^ 128u, norm_part(par ^ 1));
       gam_part(par)[pc] = g2.x + g2.y;
       if constexpr (QJL) sm100::tmem_wait_st();
       prev_norm = nrm;
       prev_row = grow;
     }
     sm100::tc_fence_before();
-    failed = __syncthreads_or(!ok || ifail) != 0;
+    failed = sm100::named_barrier_or(1, kThreadsAll, !ok);
+    if (failed) break;
+  }
+  else for (; it < nloc && !failed; ++it) {
+    const int par = it & 1;
+    const uint32_t ucol = par ? 128u : 0u;
+    failed = sm100::named_barrier_or(1, kThreadsAll, ifail);
     if (failed) break;
     // ---- (e) control thread: QJL projection of this tile, then the rotation two tiles ahead
     if (ctl) {
