@@ -992,14 +992,18 @@ struct EncGSmem {
 }  // namespace
 
 template <int D, int W, int RP, int SRCW>
-__global__ void __launch_bounds__(128 * (D / 32) + 32, 1)
+// d = 32: two CTAs per SM (one warp group each, 128 TMEM columns, under half
+// the shared memory), so that one CTA's waits overlap the other's work
+__global__ void __launch_bounds__(128 * (D / 32) + 32, D == 32 ? 2 : 1)
 k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   constexpr int P = D / 32;
   constexpr int L = 1 << W;
   constexpr int HALF = L / 2;
   constexpr int NB = SRCW / 64;      // TMA boxes of 64 columns
   constexpr int kCompute = 128 * P;  // compute threads; one more warp issues the copies and MMAs
-  constexpr uint32_t kColU0 = 0, kColZ = 256, kColA = 384;  // U double buffer, QJL accumulator, QJL A operand
+  // TMEM: U double buffer, QJL accumulator, QJL A operand, kColStep columns apart
+  constexpr uint32_t kColStep = D == 32 ? 32u : 128u, kTmemCols = D == 32 ? 128u : 512u;
+  constexpr uint32_t kColU0 = 0, kColU1 = kColStep, kColZ = 2 * kColStep, kColA = 3 * kColStep;
   using SM = EncGSmem<D, RP, SRCW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1024,7 +1028,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
     sm100::prefetch_tmap(&xmap);
   }
   if (tid < 32) {
-    sm100::tmem_alloc(sTmem, 512);
+    sm100::tmem_alloc(sTmem, kTmemCols);
     sm100::tmem_relinquish();
   }
 #pragma unroll
@@ -1178,7 +1182,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
       if (ctl) {
         pend_full = false;
         sm100::tc_fence_after();
-        if (nloc > 1) issue_rot(1, 128u);
+        if (nloc > 1) issue_rot(1, kColU1);
         if (nloc > 2) {
           issue_tma(first + 2 * stride, ntma);
           pend_full = true;
@@ -1204,7 +1208,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   for (; it < nloc && !failed; ++it) {
     const int t = first + it * stride;
     const int par = it & 1;
-    const uint32_t ucol = par ? 128u : 0u;
+    const uint32_t ucol = par ? kColU1 : kColU0;
     const int64_t grow = (int64_t)t * kRows + row;
     bool ok = true;
     if (compute) {
@@ -1286,7 +1290,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
         ok = sm100::mbar_wait(&bars[1], ph_rot, p.err, 64) && ok;
         ph_rot ^= 1u;
         sm100::tc_fence_after();
-        row_partial(ucol ^ 128u, norm_part(par ^ 1));
+        row_partial(par ? kColU0 : kColU1, norm_part(par ^ 1));
       }
       gam_part(par)[pc] = g2.x + g2.y;
       sm100::tmem_wait_st();
@@ -1332,7 +1336,7 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   }
   sm100::tc_fence_before();
   __syncthreads();
-  if (tid < 32) sm100::tmem_dealloc(tmem, 512);
+  if (tid < 32) sm100::tmem_dealloc(tmem, kTmemCols);
 }
 
 namespace {
@@ -1354,16 +1358,19 @@ tq_status launch_tcg(const void *x, int64_t n, int64_t ldx, const EncTCParams &p
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // at least half the SM's shared memory, so that one CTA (which takes all of
-  // TMEM) runs per SM
-  const int smem = std::max(EncGSmem<D, RP, SRCW>::kTotal, max_smem / 2 + 1024);
+  // d > 32: at least half the SM's shared memory, so that one CTA (which
+  // takes all of TMEM) runs per SM; d = 32: two CTAs per SM
+  const int per_sm = D == 32 ? 2 : 1;
+  const int smem = D == 32 ? EncGSmem<D, RP, SRCW>::kTotal : std::max(EncGSmem<D, RP, SRCW>::kTotal, max_smem / 2 + 1024);
   if (smem > max_smem) return TQ_ERR_UNSUPPORTED;
   EncTCParams pp = prm;
   pp.ntiles = (int)((n + kRows - 1) / kRows);
   auto kern = k_encode_tcg<D, W, RP, SRCW>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TQ_ERR_CUDA;
-  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32) + 32, smem, st>>>(map, pp);
+  if (D == 32 && cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  kern<<<std::min(pp.ntiles, sms * per_sm), 128 * (D / 32) + 32, smem, st>>>(map, pp);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
