@@ -58,7 +58,7 @@ CSRC = os.path.join(ROOT, "online_vector_quantization_tq_b200", "csrc")
 TRAFFIC = {
     # kernel@workload: (source file, digest, bytes per launch, the capture)
     "k_encode_tc2@kv": ("tq_encode_tc.cu", "43260117e29fed2c", 326731008, "kv workload, launch 4, ncu --set full"),
-    "k_score_tc@kv": ("tq_score_tc.cu", "f3d48b916b85d13a", 79352832, "kv workload, launch 4, ncu --set full"),
+    "k_score_tc@kv": ("tq_score_tc.cu", "605075399fb8a731", 79352832, "kv workload, launch 4, ncu --set full"),
     "k_attend_split@decode_attend": ("tq_attend.cu", "92d847b55e84b554", 615426816, "decode_attend workload, launch 3, ncu --set full"),
 }
 

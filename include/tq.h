@@ -275,6 +275,41 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups,
                    int64_t keys_per_group, float *out, int accumulate,
                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---------------------------------------------------------------- score in two halves
+ * tq_score split at the point where the queries and the keys meet (blog 四:
+ * the query is rotated and projected once, then scored against every packed
+ * key).  Together the two calls compute exactly what tq_score computes, with
+ * the same kernels and the same logits bit for bit, when the keys are 16-byte
+ * aligned (tq_encode's outputs are).  The query half depends on the queries
+ * only, so it may run on another stream while the keys are still being
+ * encoded, or once for several key sets.
+ *
+ * tq_score_prepare: the query half.  Arguments as tq_score's (y, groups, G,
+ *   ldy, ychan); writes the prepared queries into `workspace` (at least
+ *   tq_score_workspace_bytes(q, groups*G) bytes, 16-byte aligned).  For
+ *   d <= 128 that is the scorer's full query operand (the rotated query y~ and
+ *   its projection p = S y~, as 16-bit fixed-point limbs with their scales);
+ *   for d > 128, y~ and p in fp32 (the scoring GEMM builds its fp16 pieces).
+ * tq_score_prepared: the key half.  Arguments as tq_score's (codes, signs,
+ *   norms, keys_per_group, out, accumulate), with groups and G equal to the
+ *   prepare call's and the workspace it wrote, unchanged since.  codes and
+ *   signs must be 16-byte aligned (4-byte for quantizers that score on the CUDA
+ *   cores: d > 128 without the tensor-core route, or G > 48), else
+ *   TQ_ERR_ALIGNMENT.  For d > 128 the call also uses the workspace's scratch
+ *   region (the decoded-key chunk): two such calls must not share a workspace
+ *   at the same time.
+ * Ownership and errors as tq_score; both calls are asynchronous on `stream`,
+ * and the caller orders the prepare before the prepared call when they are on
+ * different streams. */
+tq_status tq_score_prepare(const tq_quantizer *q, const float *y, int64_t groups,
+                           int64_t G, int64_t ldy, const int32_t *ychan,
+                           void *workspace, size_t workspace_bytes, void *stream);
+tq_status tq_score_prepared(const tq_quantizer *q, int64_t groups, int64_t G,
+                            const void *codes, const void *signs,
+                            const float *norms, int64_t keys_per_group,
+                            float *out, int accumulate, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
 /* ---------------------------------------------------------------- score, no allocation
  * tq_score_noalloc: the same scores as tq_score, for callers that cannot hand
  * the library a workspace.  (No counterpart in the TurboQuant pages; this is

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         "tq_prepare_queries": (i32, [vp, vp, i64, i64, vp, i64, vp, vp, vp]),
         "tq_score_workspace_bytes": (sz, [vp, i64]),
         "tq_score": (i32, [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp, i32, vp, sz, vp]),
+        "tq_score_prepare": (i32, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "tq_score_prepared": (i32, [vp, i64, i64, vp, vp, vp, i64, vp, i32, vp, sz, vp]),
         "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
         "tq_topk": (i32, [vp, vp, i64, i64, vp, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
         "tq_score_noalloc": (i32, [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp, i32, vp]),
@@ -267,6 +269,31 @@ def tq_score(q: Quantizer, y: torch.Tensor, groups: int, G: int, enc: Encoded, k
     _check("tq_score", lib().tq_score(
         q.handle, _ptr(y), groups, G, _ld(y), _ptr(ychan), _ptr(enc.codes), _ptr(enc.signs), _ptr(enc.norms),
         keys_per_group, _ptr(out), int(bool(accumulate)), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def tq_score_prepare(q: Quantizer, y: torch.Tensor, groups: int, G: int, workspace: torch.Tensor | None = None,
+                     ychan: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Query half of tq_score: writes the prepared queries into `workspace`
+    (allocated when None) and returns it, for tq_score_prepared."""
+    if workspace is None:
+        workspace = score_workspace(q, groups * G, y.device)
+    _check("tq_score_prepare", lib().tq_score_prepare(
+        q.handle, _ptr(y), groups, G, _ld(y), _ptr(ychan), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return workspace
+
+
+def tq_score_prepared(q: Quantizer, groups: int, G: int, enc: Encoded, keys_per_group: int,
+                      workspace: torch.Tensor, out: torch.Tensor | None = None, accumulate: bool = False,
+                      stream=None) -> torch.Tensor:
+    """Key half of tq_score against the queries tq_score_prepare wrote into
+    `workspace`."""
+    enc.check()
+    if out is None:
+        out = torch.empty((groups * G, keys_per_group), dtype=torch.float32, device=enc.codes.device)
+    _check("tq_score_prepared", lib().tq_score_prepared(
+        q.handle, groups, G, _ptr(enc.codes), _ptr(enc.signs), _ptr(enc.norms), keys_per_group, _ptr(out),
+        int(bool(accumulate)), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
 
 

@@ -232,6 +232,80 @@ tq_status tq_score(const tq_quantizer *q, const float *y, int64_t groups, int64_
                   keys_per_group, accumulate, s);
 }
 
+// The scoring route for (q, G) when the keys are 16-byte aligned; the query
+// half (tq_score_prepare) and the key half (tq_score_prepared) take the same one.
+enum ScorePath { kPathTcY, kPathTc, kPathDense, kPathV1 };
+static ScorePath score_path(const tq_quantizer *q, int64_t G) {
+  if (tc_score_y_supported(q, G)) return kPathTcY;
+  if (tc_score_supported(q, G)) return kPathTc;
+  if (dense_score_supported(q)) return kPathDense;
+  return kPathV1;
+}
+
+tq_status tq_score_prepare(const tq_quantizer *q, const float *y, int64_t groups, int64_t G, int64_t ldy,
+                           const int32_t *ychan, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!q || groups < 0 || G < 0) return TQ_ERR_INVALID_ARG;
+  const int64_t nq = groups * G;
+  bool empty = false;
+  tq_status st = check_rows(q, y, TQ_F32, nq, ldy, ychan, G > 0 ? G : 1, &empty);
+  if (st != TQ_OK || empty || nq == 0) return st;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < tq_score_workspace_bytes(q, nq))
+    return TQ_ERR_WORKSPACE;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ScoreLayout L = score_layout(q, nq);
+  char *ws = static_cast<char *>(workspace);
+  float *ytil = reinterpret_cast<float *>(ws + L.ytil);
+  float *p = reinterpret_cast<float *>(ws + L.p);
+  RowSource src{y, ldy, ychan, G, q->d, 0};
+  const ScorePath path = score_path(q, G);
+  if (path == kPathTcY)
+    return tc_score_y_queries(q, src, groups, G, reinterpret_cast<int8_t *>(ws + L.qop),
+                              reinterpret_cast<float4 *>(ws + L.qsc), s);
+  st = v1_prepare_queries(q, src, nq, ytil, p, s);
+  if (st != TQ_OK || path != kPathTc) return st;
+  return tc_score_queries(q, ytil, p, groups, G, reinterpret_cast<int8_t *>(ws + L.qop),
+                          reinterpret_cast<float4 *>(ws + L.qsc), s);
+}
+
+tq_status tq_score_prepared(const tq_quantizer *q, int64_t groups, int64_t G, const void *codes,
+                            const void *signs, const float *norms, int64_t keys_per_group, float *out,
+                            int accumulate, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!q || groups < 0 || G < 0 || keys_per_group < 0) return TQ_ERR_INVALID_ARG;
+  if (q->device < 0) return TQ_ERR_UNSUPPORTED;  // host-only quantizer
+  const int64_t nq = groups * G;
+  if (!codes || (!signs && q->m > 0) || !norms || !out) return TQ_ERR_INVALID_ARG;
+  const ScorePath path = score_path(q, G);
+  const int key_align = path == kPathV1 ? 4 : 16;
+  if (!aligned(codes, key_align) || !aligned(signs, key_align) || !aligned(norms, 8) || !aligned(out, 4))
+    return TQ_ERR_ALIGNMENT;
+  if (nq == 0 || keys_per_group == 0) return TQ_OK;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < tq_score_workspace_bytes(q, nq))
+    return TQ_ERR_WORKSPACE;
+  DeviceGuard g(q->device);
+  if (!g.ok) return TQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ScoreLayout L = score_layout(q, nq);
+  char *ws = static_cast<char *>(workspace);
+  const float *ytil = reinterpret_cast<const float *>(ws + L.ytil);
+  const float *p = reinterpret_cast<const float *>(ws + L.p);
+  const int64_t kpg = keys_per_group;
+  switch (path) {
+    case kPathTcY:
+    case kPathTc:
+      return tc_score_keys(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, kpg, accumulate,
+                           reinterpret_cast<const int8_t *>(ws + L.qop), reinterpret_cast<const float4 *>(ws + L.qsc),
+                           s);
+    case kPathDense:
+      // the dense path's own scratch follows the prepared queries in the workspace
+      return dense_score(q, ytil, p, nq, G, kpg, 0, kpg, codes, signs, norms, out, kpg, accumulate, ws + L.dense,
+                         L.total - L.dense, s);
+    default:
+      return v1_score(q, ytil, p, nq, G, kpg, 0, kpg, codes, signs, norms, out, kpg, accumulate, s);
+  }
+}
+
 }  // extern "C"
 
 namespace {

@@ -91,15 +91,27 @@ bool tc2_encode_supported(const tq_quantizer *q, int dtype, bool gather);
 tq_status tc2_encode(const tq_quantizer *q, const void *x, int64_t n, int64_t ldx, void *codes, void *signs,
                      float *norms, int64_t out_stride, cudaStream_t st);
 
+// Integer tensor-core scorer (d <= 128), in two halves: the query operand
+// and scales (qop, qsc) from the queries alone, then the scores of packed
+// keys against them.  tc_score and tc_score_y run both halves.
 bool tc_score_supported(const tq_quantizer *q, int64_t G);
-// tq_score from raw queries for Hadamard d = 32, 64, 128: query preparation
-// and the operand fused in one kernel (bit-identical to tc_score after
-// v1_prepare_queries).
+// the query half from raw queries for Hadamard d = 32, 64, 128: query
+// preparation and the operand fused in one kernel (bit-identical to
+// tc_score_queries after v1_prepare_queries)
 bool tc_score_y_supported(const tq_quantizer *q, int64_t G);
+tq_status tc_score_y_queries(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int8_t *qop,
+                             float4 *qsc, cudaStream_t st);
 tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int64_t kpg,
                      const void *codes, const void *signs, const float *norms, float *out, int64_t ldo,
                      int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st);
 size_t tc_score_qop_bytes(const tq_quantizer *q, int64_t groups, int64_t G);
+// the query half from prepared queries (y~, p)
+tq_status tc_score_queries(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
+                           int8_t *qop, float4 *qsc, cudaStream_t st);
+// the key half: keys [key_base, key_base + nkeys) of every group
+tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
+                        int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
+                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, cudaStream_t st);
 tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
                    int64_t kpg, int64_t key_base, int64_t nkeys, const void *codes, const void *signs,
                    const float *norms, float *out, int64_t ldo, int accumulate, int8_t *qop, float4 *qsc,

@@ -674,24 +674,24 @@ size_t tc_score_qop_bytes(const tq_quantizer *q, int64_t groups, int64_t G) {
   return (size_t)groups * N * kScoreKBytes;
 }
 
-namespace {
-tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
-                          int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
-                          int64_t ldo, int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st);
-}  // namespace
-
-tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
-                   int64_t kpg, int64_t key_base, int64_t nkeys, const void *codes, const void *signs,
-                   const float *norms, float *out, int64_t ldo, int accumulate, int8_t *qop, float4 *qsc,
-                   cudaStream_t st) {
+tq_status tc_score_queries(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
+                           int8_t *qop, float4 *qsc, cudaStream_t st) {
   const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   const int64_t nq = groups * G;
   if (cudaMemsetAsync(qop, 0, tc_score_qop_bytes(q, groups, G), st) != cudaSuccess) return TQ_ERR_CUDA;
   k_query_operand<<<(unsigned)nq, 128, 0, st>>>(ytil, pq, q->d, q->m, q->w, G, N, q->score_cexp, q->kt.qjl_scale,
                                                 qop, qsc);
-  if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
-  return tc_score_launch(q, groups, G, kpg, key_base, nkeys, codes, signs, norms, out, ldo, accumulate, qop, qsc,
-                         st);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
+                   int64_t kpg, int64_t key_base, int64_t nkeys, const void *codes, const void *signs,
+                   const float *norms, float *out, int64_t ldo, int accumulate, int8_t *qop, float4 *qsc,
+                   cudaStream_t st) {
+  const tq_status r = tc_score_queries(q, ytil, pq, groups, G, qop, qsc, st);
+  if (r != TQ_OK) return r;
+  return tc_score_keys(q, groups, G, kpg, key_base, nkeys, codes, signs, norms, out, ldo, accumulate, qop, qsc,
+                       st);
 }
 
 bool tc_score_y_supported(const tq_quantizer *q, int64_t G) {
@@ -699,9 +699,8 @@ bool tc_score_y_supported(const tq_quantizer *q, int64_t G) {
          (q->d == 32 || q->d == 64 || q->d == 128) && q->kt.diag_bits;
 }
 
-tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int64_t kpg,
-                     const void *codes, const void *signs, const float *norms, float *out, int64_t ldo,
-                     int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st) {
+tq_status tc_score_y_queries(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int8_t *qop,
+                             float4 *qsc, cudaStream_t st) {
   const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   const unsigned nq = (unsigned)(groups * G);
   switch (q->d) {
@@ -710,14 +709,20 @@ tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups
     case 128: k_prep_operand<128><<<nq, 128, 0, st>>>(q->kt, src, G, N, q->score_cexp, qop, qsc); break;
     default: return TQ_ERR_UNSUPPORTED;
   }
-  if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
-  return tc_score_launch(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, ldo, accumulate, qop, qsc, st);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
-namespace {
-tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
-                          int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
-                          int64_t ldo, int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st) {
+tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int64_t kpg,
+                     const void *codes, const void *signs, const float *norms, float *out, int64_t ldo,
+                     int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st) {
+  const tq_status r = tc_score_y_queries(q, src, groups, G, qop, qsc, st);
+  if (r != TQ_OK) return r;
+  return tc_score_keys(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, ldo, accumulate, qop, qsc, st);
+}
+
+tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
+                        int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
+                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, cudaStream_t st) {
   const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   ScoreTCParams prm{};
   prm.d = q->d;
@@ -800,6 +805,5 @@ tq_status tc_score_launch(const tq_quantizer *q, int64_t groups, int64_t G, int6
 #undef TQ_SC
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
-}  // namespace
 
 }  // namespace tq

@@ -676,3 +676,43 @@ def test_attend_argument_checks(tq):
         tq.tq_attend(qv, logits, 1, 4, venc, 256, float("nan"))
     out = tq.tq_attend(qv, logits, 1, 4, venc, 256, 0.1)  # zero values: zero output
     assert torch.all(out == 0)
+
+
+@pytest.mark.parametrize("d,b,rot,G,mse", [(128, 4, "auto", 4, False), (96, 3, "auto", 4, False),
+                                           (256, 3, "hadamard", 4, False), (128, 3, "auto", 60, False),
+                                           (64, 2, "auto", 3, True)])
+def test_score_in_two_halves(tq, d, b, rot, G, mse):
+    """tq_score_prepare (on a side stream) then tq_score_prepared gives tq_score's
+    logits bit for bit on every scoring route: the fused Hadamard query operand
+    (d = 128), the separate operand (d = 96), the dense GEMM (d = 256), the CUDA
+    cores (G = 60 > 48) and TurboQuant-MSE keys (m = 0).  One preparation serves
+    two key sets; accumulate adds onto the output; the first case is also checked
+    against the oracle."""
+    groups, kpg = 3, 1000  # a ragged last tile
+    rng = np.random.default_rng(d + G)
+    x = rng.standard_normal((2, groups * kpg, d)).astype(np.float32)
+    y = rng.standard_normal((groups * G, d)).astype(np.float32)
+    q = tq.tq_codebook_mse(d, b, seed=0, rotation=rot) if mse else tq.tq_codebook(d, b, seed=0, rotation=rot)
+    encs = [tq.tq_encode(q, dev(x[i])) for i in range(2)]
+    yd = dev(y)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        ws = tq.tq_score_prepare(q, yd, groups, G, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    for enc in encs:
+        ref = tq.tq_score(q, yd, groups, G, enc, kpg)
+        got = tq.tq_score_prepared(q, groups, G, enc, kpg, ws)
+        assert torch.equal(got, ref)
+        tq.tq_score_prepared(q, groups, G, enc, kpg, ws, out=got, accumulate=True)
+        assert torch.equal(got, ref + ref)
+    if d == 128 and not mse:
+        t = tables(d, b, rot)
+        rep = check_encode(*host(encs[0]), x[0], t)
+        s = tq.tq_score_prepared(q, groups, G, encs[0], kpg, ws).cpu().numpy()
+        yt = o.prepare_query(y, t)
+        for g in range(groups):
+            rows, keys = slice(g * G, (g + 1) * G), slice(g * kpg, (g + 1) * kpg)
+            r = {k: v[keys] for k, v in rep.ref.items()}
+            check_scores(s[rows], o.score(yt[0][rows], yt[1][rows], r, t), r["norm"],
+                         np.linalg.norm(y[rows], axis=1), d, rep.skip_rows[keys])

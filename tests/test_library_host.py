@@ -145,3 +145,18 @@ def test_encoded_views_must_be_contiguous(tq):
     tq.binding.Encoded(enc.codes[8:], enc.signs[8:], enc.norms[8:]).check()  # a row offset is fine
     with pytest.raises(ValueError):
         tq.binding.Encoded(enc.codes[::4], enc.signs[::4], enc.norms[::4]).check()
+
+
+def test_split_score_refuses_bad_arguments_before_any_launch(tq):
+    """tq_score_prepare / tq_score_prepared validate on the host: a missing or
+    host-only quantizer, missing key arrays and a short workspace are refused
+    without touching a pointer (no GPU needed)."""
+    q = tq.tq_codebook_host(128, 4)
+    L = tq.lib()
+    fake = ctypes.c_void_p(0x1000)
+    assert L.tq_score_prepare(None, fake, 2, 4, 128, None, fake, 1 << 20, None) == 1
+    assert L.tq_score_prepare(q.handle, fake, 2, 4, 128, None, fake, 1 << 20, None) == 2
+    assert L.tq_score_prepare(q.handle, fake, -1, 4, 128, None, fake, 1 << 20, None) == 1
+    assert L.tq_score_prepared(None, 2, 4, fake, fake, fake, 16, fake, 0, fake, 1 << 20, None) == 1
+    assert L.tq_score_prepared(q.handle, 2, 4, fake, fake, fake, 16, fake, 0, fake, 1 << 20, None) == 2
+    assert L.tq_score_prepared(q.handle, 2, 4, fake, fake, fake, -5, fake, 0, fake, 1 << 20, None) == 1
