@@ -52,20 +52,24 @@ CSRC = os.path.join(ROOT, "online_vector_quantization_tq_b200", "csrc")
 
 # DRAM bytes (read + write) per launch counted by ncu for a kernel on one
 # workload ("kernel@workload"), with the SHA-256 (first 16 hex digits) of the
-# source file it was built from at the time of the capture.  A figure is
-# reported only for that workload and while the source is unchanged;
-# otherwise the roofline's traffic is null.
+# source file it was built from and of every header of the library, at the
+# time of the capture.  A figure is reported only for that workload and while
+# those sources are unchanged; otherwise the roofline's traffic is null.
 TRAFFIC = {
     # kernel@workload: (source file, digest, bytes per launch, the capture)
-    "k_encode_tc2@kv": ("tq_encode_tc.cu", "43260117e29fed2c", 326731008, "kv workload, launch 4, ncu --set full"),
-    "k_score_tc@kv": ("tq_score_tc.cu", "605075399fb8a731", 79352832, "kv workload, launch 4, ncu --set full"),
-    "k_attend_split@decode_attend": ("tq_attend.cu", "92d847b55e84b554", 615426816, "decode_attend workload, launch 3, ncu --set full"),
+    "k_encode_tc2@kv": ("tq_encode_tc.cu", "ea25e4b8464cdc63", 326488576, "kv workload, launch 4, ncu --set full"),
+    "k_score_tc@kv": ("tq_score_tc.cu", "9f4d14f7a3b1cb30", 80218880, "kv workload, launch 4, ncu --set full"),
+    "k_attend_split@decode_attend": ("tq_attend.cu", "d0b6ad53ba88c5bc", 614982656, "decode_attend workload, launch 3, ncu --set full"),
 }
 
 
 def _source_digest(fname: str) -> str:
-    with open(os.path.join(CSRC, fname), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Digest of a kernel's source file and of every header it may include."""
+    h = hashlib.sha256()
+    for name in [fname] + sorted(n for n in os.listdir(CSRC) if n.endswith((".h", ".cuh"))):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str, workload=None):

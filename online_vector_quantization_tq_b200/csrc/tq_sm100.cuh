@@ -344,14 +344,28 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
 // Copy a row-major 16-bit [rows][D] matrix from global memory into a 64-byte
 // swizzled K-major operand (D/32 blocks of rows x 64 B), all threads of the
 // block taking 16-byte chunks in turn.
+// Each thread loads four chunks before storing any, so that a block's
+// staging takes about one memory round trip per four chunks per thread rather
+// than one per chunk.
 template <int D>
 __device__ void stage_kmajor(uint8_t *dst, const uint16_t *src, int rows) {
+  constexpr int kBatch = 4;
   const int chunks = rows * (D / 8);
-  for (int i = threadIdx.x; i < chunks; i += blockDim.x) {
-    const int r = i / (D / 8), c8 = i % (D / 8);  // 8-element chunk index along K
-    const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * D + c8 * 8);
-    const int blk = c8 / 4, ch = c8 % 4;
-    *reinterpret_cast<uint4 *>(dst + (size_t)blk * rows * 64 + sw64_offset(r, ch)) = v;
+  for (int i0 = threadIdx.x; i0 < chunks; i0 += kBatch * blockDim.x) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      if (i < chunks) v[u] = *reinterpret_cast<const uint4 *>(src + (size_t)(i / (D / 8)) * D + (i % (D / 8)) * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      if (i < chunks) {
+        const int r = i / (D / 8), c8 = i % (D / 8);  // 8-element chunk index along K
+        *reinterpret_cast<uint4 *>(dst + (size_t)(c8 / 4) * rows * 64 + sw64_offset(r, c8 % 4)) = v[u];
+      }
+    }
   }
 }
 
