@@ -62,6 +62,7 @@ k_query_operand(const float *ytil, const float *p, int d, int m, int w, int64_t 
   // byte k of operand row n sits where the 128-byte-swizzled K-major tile
   // (three 128-byte K atoms of N rows) keeps it in shared memory
   auto at = [N](int n, int k) { return (k / 128) * (N * 128) + sm100::sw128_offset(n, (k % 128) / 16) + k % 16; };
+  sm100::pdl_launch_dependents();  // the scorer waits for this kernel only where it reads qop and qsc
   const int64_t qrow = blockIdx.x;
   const int64_t g = qrow / G, ql = qrow % G;
   const float *yr = ytil + qrow * d;
@@ -134,6 +135,7 @@ k_prep_operand(KernelTables kt, RowSource src, int64_t G, int N, int cexp, int8_
   __shared__ __align__(16) int8_t stg[kColsPerQuery][kScoreKBytes];
   const int64_t row = blockIdx.x;
   const int j = threadIdx.x;
+  sm100::pdl_launch_dependents();  // the scorer waits for this kernel only where it reads qop and qsc
   for (int i = j; i < kColsPerQuery * kScoreKBytes / 16; i += D) reinterpret_cast<uint4 *>(&stg[0][0])[i] = make_uint4(0, 0, 0, 0);
   float x = src.at(row, j);
 #pragma unroll
@@ -391,7 +393,8 @@ k_score_tc(const ScoreTCParams p) {
     return sm100::mbar_wait_abort(&bars[bar], parity, sAbort, p.err, code);
   };
   // state the teardown needs
-  int64_t issued = 0;  // stages issued (load warp)
+  int64_t issued = 0;  // tiles the load warp has passed (their key stages and query operands issued)
+  int64_t pre = 0;     // key stages issued ahead of the first query operand (load warp)
   int b_loaded = 0;    // query operands issued (load warp)
   int mma_issued = 0;  // tiles whose MMAs this thread issued (MMA issuers)
 
@@ -475,6 +478,7 @@ k_score_tc(const ScoreTCParams p) {
     }
   } else if (warp < kMmaWarp) {
     // ------------------------------------------------------------ epilogue
+    sm100::pdl_wait();  // the query scales (qsc) are final from here on
     const int quarter = warp % 4, eh = (warp - kExpWarps) / 4, row = 32 * quarter + lane;
     const int q_half = (int)((p.G + 1) / 2);
     const int q_lo = eh ? q_half : 0, q_hi = eh ? (int)p.G : q_half;
@@ -599,6 +603,27 @@ k_score_tc(const ScoreTCParams p) {
     }
   } else if (lane == 0) {
     // ------------------------------------------------------------ copies
+    // key rows of tile jt into ring slot jt % NS (the slot is free)
+    auto issue_keys = [&](int jt, const TileWalk &w) {
+      const int slot = jt % NS;
+      const int64_t kin0 = w.tin * 128;
+      const int64_t key0 = w.g * p.kpg + p.key_base + kin0;
+      const int64_t left = p.nkeys - kin0;
+      const int rows = left < 128 ? (int)left : 128;
+      uint8_t *st = sStage + slot * SM::kStageBytes;
+      const uint32_t cb = rows * CW * 4, sb = p.m > 0 ? rows * NG * 4 : 0;
+      sm100::mbar_expect_tx(&bars[SM::kFull + slot], cb + sb);
+      sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
+      if (sb) sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
+    };
+    // The key stages that fit in the ring go first: the keys were written
+    // before the query preparation started, so they need no wait; the query
+    // operands come from that kernel, which may still be running.
+    if constexpr (BULK) {
+      TileWalk tp(t0, tpg);
+      for (; pre < n_it && pre < NS; ++pre, tp.advance(1)) issue_keys((int)pre, tp);
+    }
+    sm100::pdl_wait();  // the query operands (qop) are final from here on
     TileWalk tw(t0, tpg);
     for (; issued < n_it; ++issued, tw.advance(1)) {
       const int j = (int)(tw.g - g0);
@@ -609,17 +634,10 @@ k_score_tc(const ScoreTCParams p) {
         ++b_loaded;
       }
       if constexpr (BULK) {
-        const int jt = (int)issued, slot = jt % NS;
-        if (jt >= NS && !wait(SM::kEmpty + slot, (uint32_t)((jt / NS - 1) & 1), 28)) break;
-        const int64_t kin0 = tw.tin * 128;
-        const int64_t key0 = tw.g * p.kpg + p.key_base + kin0;
-        const int64_t left = p.nkeys - kin0;
-        const int rows = left < 128 ? (int)left : 128;
-        uint8_t *st = sStage + slot * SM::kStageBytes;
-        const uint32_t cb = rows * CW * 4, sb = p.m > 0 ? rows * NG * 4 : 0;
-        sm100::mbar_expect_tx(&bars[SM::kFull + slot], cb + sb);
-        sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
-        if (sb) sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
+        const int jt = (int)issued;
+        if (jt < pre) continue;  // issued ahead
+        if (!wait(SM::kEmpty + jt % NS, (uint32_t)((jt / NS - 1) & 1), 28)) break;
+        issue_keys(jt, tw);
       }
     }
   }
@@ -634,7 +652,8 @@ k_score_tc(const ScoreTCParams p) {
     // copies issued but possibly not consumed: the last p.nstages key stages
     // and the last two query operands
     if constexpr (BULK) {
-      for (int64_t j = issued > NS ? issued - NS : 0; j < issued; ++j)
+      const int64_t kst = issued > pre ? issued : pre;  // key stages issued
+      for (int64_t j = kst > NS ? kst - NS : 0; j < kst; ++j)
         sm100::mbar_wait(&bars[SM::kFull + j % NS], (uint32_t)((j / NS) & 1), p.err, 31);
     }
     for (int j = b_loaded > 2 ? b_loaded - 2 : 0; j < b_loaded; ++j)
@@ -778,12 +797,26 @@ tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = std::min<int64_t>(prm.ntiles, (int64_t)sms);
   if (grid <= 0) return TQ_OK;
+  // Programmatic dependent launch: after the query-side kernel (which lets
+  // its dependents start at once) the scorer sets up and loads keys while
+  // that kernel still runs; its threads wait for it where they read qop and
+  // qsc.  After any other kernel it starts as usual.
+  cudaLaunchAttribute pdl{};
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kScoreThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
 #define TQ_SC(WW, NGG)                                                                                   \
   {                                                                                                      \
     auto kern = bulk ? k_score_tc<WW, NGG, true> : k_score_tc<WW, NGG, false>;                           \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
       return TQ_ERR_CUDA;                                                                                \
-    kern<<<(unsigned)grid, kScoreThreads, smem, st>>>(prm);                                                        \
+    if (cudaLaunchKernelEx(&cfg, kern, prm) != cudaSuccess) return TQ_ERR_CUDA;                          \
     break;                                                                                               \
   }
 #define TQ_SC_NG(WW)                     \

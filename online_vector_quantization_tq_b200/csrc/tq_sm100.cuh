@@ -108,6 +108,19 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  A kernel that calls pdl_launch_dependents
+// lets the next kernel of its stream, if that one was launched with
+// programmatic stream serialization, start before it has finished; the
+// dependent kernel's threads call pdl_wait before they read anything the
+// first kernel writes (it returns once that kernel has completed and its
+// writes are visible).  Without the launch attribute, or after a kernel that
+// never calls pdl_launch_dependents, the dependent kernel starts after the
+// previous one as usual and pdl_wait returns at once.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ TMA
 // 2-D tiled load of box {c0 (inner), c1} into shared memory, completing on
 // `bar` (transaction bytes must have been announced with mbar_expect_tx).
