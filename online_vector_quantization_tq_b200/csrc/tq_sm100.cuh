@@ -421,3 +421,26 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 }  // namespace sm100
 }  // namespace tq
+
+namespace tq {
+// Host: launch configuration with programmatic stream serialization.  The
+// kernel may start while the previous kernel of its stream is still running,
+// once that kernel calls pdl_launch_dependents (every CTA) or finishes; the
+// kernel calls pdl_wait before it touches memory the previous one may write.
+struct PdlLaunch {
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t cfg;
+  PdlLaunch(unsigned grid, unsigned block, size_t smem, cudaStream_t st) : attr{}, cfg{} {
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+  }
+  PdlLaunch(const PdlLaunch &) = delete;  // cfg points at attr
+  PdlLaunch &operator=(const PdlLaunch &) = delete;
+};
+}  // namespace tq
