@@ -187,8 +187,12 @@ class Phases:
     def __init__(self, torch, stream):
         self.torch, self.stream = torch, stream
         self.ev = {}
+        self.enabled = True
 
     def __call__(self, name, fn):
+        if not self.enabled:
+            fn()
+            return
         a = self.torch.cuda.Event(enable_timing=True)
         b = self.torch.cuda.Event(enable_timing=True)
         a.record(self.stream)
@@ -205,12 +209,15 @@ class Phases:
 
 def timed_steps(torch, dev, stream, step, steps, warmup, phases=None, clock=None):
     """W untimed warm-up steps, then K timed steps bracketed by synchronize;
-    returns ms per step (CUDA events on `stream`)."""
+    returns ms per step (CUDA events on `stream`).  The timed steps run with
+    `phases` off: an event between two kernels would stop the second from
+    starting in the first one's tail.  With `phases`, K more steps then record
+    the per-phase events."""
+    if phases is not None:
+        phases.enabled = False
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
-    if phases is not None:
-        phases.clear()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -218,7 +225,14 @@ def timed_steps(torch, dev, stream, step, steps, warmup, phases=None, clock=None
         step()
     t1.record(stream)
     torch.cuda.synchronize(dev)
-    return t0.elapsed_time(t1) / steps
+    ms = t0.elapsed_time(t1) / steps
+    if phases is not None:
+        phases.enabled = True
+        phases.clear()
+        for _ in range(steps):
+            step()
+        torch.cuda.synchronize(dev)
+    return ms
 
 
 def roofline_hbm(algo_bytes, ms, peak, kernel, unit_note, workload=None):
@@ -526,17 +540,22 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
     ph = Phases(torch, stream)
     it = [0]
 
+    # The query half of the score (tq_score_prepare: rotation, projection and
+    # operand of the 32 queries) goes first, so that the encode's set-up
+    # (launched with programmatic dependent launch) overlaps it; the key half
+    # (tq_score_prepared) follows the encode.
     def step(record=True):
         i = it[0]
         it[0] += 1
         e_w, e_r = encs[i % 2], encs[(i + 1) % 2]
         if record:
+            ph("prepare", lambda: tq.tq_score_prepare(q, y_dev, groups, G, workspace=ws, stream=stream))
             ph("encode", lambda: tq.tq_encode(q, x_dev, out=e_w, stream=stream))
-            ph("score", lambda: tq.tq_score(q, y_dev, groups, G, e_r, kpg, out=logits, workspace=ws,
-                                            stream=stream))
+            ph("score", lambda: tq.tq_score_prepared(q, groups, G, e_r, kpg, ws, out=logits, stream=stream))
         else:
+            tq.tq_score_prepare(q, y_dev, groups, G, workspace=ws, stream=stream)
             tq.tq_encode(q, x_dev, out=e_w, stream=stream)
-            tq.tq_score(q, y_dev, groups, G, e_r, kpg, out=logits, workspace=ws, stream=stream)
+            tq.tq_score_prepared(q, groups, G, e_r, kpg, ws, out=logits, stream=stream)
 
     for _ in range(max(args.warmup, 3)):
         step(False)
@@ -562,8 +581,9 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
-        ph.clear()
-        ms = timed_steps(torch, dev, stream, step, args.steps, 0, phases=None)
+        # the timed steps carry no events between their kernels (an event there
+        # would stop a kernel from starting in the previous one's tail)
+        ms = timed_steps(torch, dev, stream, lambda: step(False), args.steps, 0, phases=None)
         if world > 1:
             dist.barrier()
         n1, t_end = clk.count(), time.time() + 1.0
@@ -571,6 +591,11 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
             for _ in range(max(1, int(50.0 / max(warm_ms, 1e-3)))):
                 step(False)
             torch.cuda.synchronize(dev)
+    # per-phase times from as many more steps, with events between the phases
+    ph.clear()
+    for _ in range(args.steps):
+        step(True)
+    torch.cuda.synchronize(dev)
     pm = ph.mean_ms()
     enc_ms, score_ms = pm["encode"], pm["score"]
     if world > 1:
@@ -586,10 +611,11 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
     y_stage = torch.empty_like(y_dev)
 
     def e2e_step():
-        x_stage.copy_(x_pin, non_blocking=True)
         y_stage.copy_(y_pin, non_blocking=True)
+        tq.tq_score_prepare(q, y_stage, groups, G, workspace=ws, stream=stream)
+        x_stage.copy_(x_pin, non_blocking=True)
         tq.tq_encode(q, x_stage, out=encs[0], stream=stream)
-        tq.tq_score(q, y_stage, groups, G, encs[0], kpg, out=logits, workspace=ws, stream=stream)
+        tq.tq_score_prepared(q, groups, G, encs[0], kpg, ws, out=logits, stream=stream)
         out_pin.copy_(logits, non_blocking=True)
 
     if world > 1:
@@ -620,19 +646,24 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
                                "per head x10; 32 query heads (group 4); b=4; all fp32 logits",
                    "keys_per_step_per_gpu": n, "parallelism": f"dp{world} (independent layers, no collective)",
                    "l2": "no flush: keys (256 MiB) exceed L2; two code buffers, each step scores the codes "
-                         "encoded one step earlier (>330 MB of other traffic in between)"},
+                         "encoded one step earlier (>330 MB of other traffic in between)",
+                   "step": "tq_score_prepare (the 32 queries), tq_encode (the keys), tq_score_prepared (the "
+                           "queries against the keys encoded one step earlier), on one stream with "
+                           "programmatic dependent launch between the kernels"},
         "encode_vectors_per_s": world * n / (enc_ms * 1e-3),
         "score_keys_per_s": world * n / (score_ms * 1e-3),
         "score_logits_per_s": world * n * G / (score_ms * 1e-3),
         "encode_ms": enc_ms,
         "score_ms": score_ms,
+        "prepare_ms": pm["prepare"],
         "roofline": roofline_hbm(n * enc_bytes_key, enc_ms, peak, "k_encode_tc2",
                                  f"{enc_bytes_key} B/key (256 in, 48 codes + 16 signs + 8 norms out) x {n} keys",
                                  workload="kv"),
         "score_roofline": dict(roofline_hbm(n * score_bytes_key, score_ms, peak, "k_score_tc",
                                             f"{score_bytes_key} B/key (72 in, 4 logits x 4 B out) x {n} keys",
                                             workload="kv"),
-                               note="phase time: the fused query preparation kernel + the scorer"),
+                               note="phase time: the scorer (tq_score_prepared) alone; the query preparation "
+                                    "(tq_score_prepare, prepare_ms) runs before the encode"),
         "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "keys/s",
                 "h2d_bytes_per_step": x_pin.numel() * 2 + y_pin.numel() * 4,
                 "d2h_bytes_per_step": out_pin.numel() * 4},
@@ -652,8 +683,8 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
     return line, quality
 
 
-# kernels of libtq launched per headline step: encode (1), the fused query
-# preparation with the integer scorer's query operand (1), scoring (1)
+# kernels of libtq launched per headline step: the fused query preparation
+# with the integer scorer's query operand (1), encode (1), scoring (1)
 LAUNCHES_PER_STEP = 3
 
 
