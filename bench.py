@@ -207,6 +207,13 @@ class Phases:
         return {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in self.ev.items()}
 
 
+def device_errors(tq, *qs):
+    """Raise if a kernel of these quantizers recorded an error during the steps
+    (a bounded wait that gave up): their results, and the time, would be void."""
+    for q in qs:
+        tq.tq_sync_check(q)
+
+
 def timed_steps(torch, dev, stream, step, steps, warmup, phases=None, clock=None):
     """W untimed warm-up steps, then K timed steps bracketed by synchronize;
     returns ms per step (CUDA events on `stream`).  The timed steps run with
@@ -540,22 +547,17 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
     ph = Phases(torch, stream)
     it = [0]
 
-    # The query half of the score (tq_score_prepare: rotation, projection and
-    # operand of the 32 queries) goes first, so that the encode's set-up
-    # (launched with programmatic dependent launch) overlaps it; the key half
-    # (tq_score_prepared) follows the encode.
     def step(record=True):
         i = it[0]
         it[0] += 1
         e_w, e_r = encs[i % 2], encs[(i + 1) % 2]
         if record:
-            ph("prepare", lambda: tq.tq_score_prepare(q, y_dev, groups, G, workspace=ws, stream=stream))
             ph("encode", lambda: tq.tq_encode(q, x_dev, out=e_w, stream=stream))
-            ph("score", lambda: tq.tq_score_prepared(q, groups, G, e_r, kpg, ws, out=logits, stream=stream))
+            ph("score", lambda: tq.tq_score(q, y_dev, groups, G, e_r, kpg, out=logits, workspace=ws,
+                                            stream=stream))
         else:
-            tq.tq_score_prepare(q, y_dev, groups, G, workspace=ws, stream=stream)
             tq.tq_encode(q, x_dev, out=e_w, stream=stream)
-            tq.tq_score_prepared(q, groups, G, e_r, kpg, ws, out=logits, stream=stream)
+            tq.tq_score(q, y_dev, groups, G, e_r, kpg, out=logits, workspace=ws, stream=stream)
 
     for _ in range(max(args.warmup, 3)):
         step(False)
@@ -584,6 +586,7 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
         # the timed steps carry no events between their kernels (an event there
         # would stop a kernel from starting in the previous one's tail)
         ms = timed_steps(torch, dev, stream, lambda: step(False), args.steps, 0, phases=None)
+        device_errors(tq, q)
         if world > 1:
             dist.barrier()
         n1, t_end = clk.count(), time.time() + 1.0
@@ -611,16 +614,16 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
     y_stage = torch.empty_like(y_dev)
 
     def e2e_step():
-        y_stage.copy_(y_pin, non_blocking=True)
-        tq.tq_score_prepare(q, y_stage, groups, G, workspace=ws, stream=stream)
         x_stage.copy_(x_pin, non_blocking=True)
+        y_stage.copy_(y_pin, non_blocking=True)
         tq.tq_encode(q, x_stage, out=encs[0], stream=stream)
-        tq.tq_score_prepared(q, groups, G, encs[0], kpg, ws, out=logits, stream=stream)
+        tq.tq_score(q, y_stage, groups, G, encs[0], kpg, out=logits, workspace=ws, stream=stream)
         out_pin.copy_(logits, non_blocking=True)
 
     if world > 1:
         dist.barrier()
     e2e_ms = timed_steps(torch, dev, stream, e2e_step, args.steps, max(1, args.warmup))
+    device_errors(tq, q)
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -647,23 +650,21 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
                    "keys_per_step_per_gpu": n, "parallelism": f"dp{world} (independent layers, no collective)",
                    "l2": "no flush: keys (256 MiB) exceed L2; two code buffers, each step scores the codes "
                          "encoded one step earlier (>330 MB of other traffic in between)",
-                   "step": "tq_score_prepare (the 32 queries), tq_encode (the keys), tq_score_prepared (the "
-                           "queries against the keys encoded one step earlier), on one stream with "
-                           "programmatic dependent launch between the kernels"},
+                   "step": "tq_encode (the keys), tq_score (the 32 queries against the keys encoded one "
+                           "step earlier), on one stream"},
         "encode_vectors_per_s": world * n / (enc_ms * 1e-3),
         "score_keys_per_s": world * n / (score_ms * 1e-3),
         "score_logits_per_s": world * n * G / (score_ms * 1e-3),
         "encode_ms": enc_ms,
         "score_ms": score_ms,
-        "prepare_ms": pm["prepare"],
         "roofline": roofline_hbm(n * enc_bytes_key, enc_ms, peak, "k_encode_tc2",
                                  f"{enc_bytes_key} B/key (256 in, 48 codes + 16 signs + 8 norms out) x {n} keys",
                                  workload="kv"),
         "score_roofline": dict(roofline_hbm(n * score_bytes_key, score_ms, peak, "k_score_tc",
                                             f"{score_bytes_key} B/key (72 in, 4 logits x 4 B out) x {n} keys",
                                             workload="kv"),
-                               note="phase time: the scorer (tq_score_prepared) alone; the query preparation "
-                                    "(tq_score_prepare, prepare_ms) runs before the encode"),
+                               note="phase time: the fused query preparation kernel + the scorer (which starts "
+                                    "during the preparation: programmatic dependent launch)"),
         "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "keys/s",
                 "h2d_bytes_per_step": x_pin.numel() * 2 + y_pin.numel() * 4,
                 "d2h_bytes_per_step": out_pin.numel() * 4},
@@ -683,8 +684,8 @@ def run_kv(args, rank, world, local, torch, tq, dev, stream, peak):
     return line, quality
 
 
-# kernels of libtq launched per headline step: the fused query preparation
-# with the integer scorer's query operand (1), encode (1), scoring (1)
+# kernels of libtq launched per headline step: encode (1), the fused query
+# preparation with the integer scorer's query operand (1), scoring (1)
 LAUNCHES_PER_STEP = 3
 
 
@@ -708,6 +709,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
             ph("encode", lambda: tq.tq_encode(q, x, out=enc, stream=stream))
             ph("topk", lambda: tq.tq_topk(q, y, enc, 10, workspace=ws, stream=stream))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        device_errors(tq, q)
         pm = ph.mean_ms()
         eb, sb = 512 + q.code_bytes + q.sign_bytes + 8, q.code_bytes + q.sign_bytes + 8
         rec = {"workload": "tiny: 4096 keys d=128 fp32 N(0,1), b=3, 16 queries, top-10",
@@ -748,6 +750,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
                                  tq.tq_score(qb, y, groups, G, rb, kpg, out=out, accumulate=True, ychan=rest,
                                              workspace=wsb, stream=stream)))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        device_errors(tq, qa, qb)
         pm = ph.mean_ms()
         enc_ms = pm[pa] + pm[pb]
         key_b = qa.code_bytes + qa.sign_bytes + 8 + qb.code_bytes + qb.sign_bytes + 8
@@ -788,6 +791,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
             ph("score", lambda: tq.tq_score(q, y, groups, G, encs[(i + 1) % 2], kpg, out=logits, workspace=ws,
                                             stream=stream))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        device_errors(tq, q)
         pm = ph.mean_ms()
         kb = q.code_bytes + 8
         rec = {"workload": "kv_mse: the kv workload with TurboQuant-MSE keys (b = 3 bits all to the codebook, no QJL "
@@ -832,6 +836,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
             ph("score", lambda: tq.tq_score(q, y, groups, G, encs[(i + 1) % 2], kpg, out=logits, workspace=ws,
                                             stream=stream))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        device_errors(tq, q)
         pm = ph.mean_ms()
         kb = q.code_bytes + q.sign_bytes + 8
         e = encs[0]
@@ -874,6 +879,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
             ph("append", lambda: tq.tq_encode(q, new, out=tail, out_stride=kpg, stream=stream))
             ph("score", lambda: tq.tq_score(q, y, groups, G, cache, kpg, out=out, workspace=ws, stream=stream))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        device_errors(tq, q)
         pm = ph.mean_ms()
         sb = q.code_bytes + q.sign_bytes + 8 + 4 * G
         rec = {"workload": "decode: 32 sequences x 8 KV heads = 256 caches x 32768 keys, d=128, bf16, b=3; step = "
@@ -920,6 +926,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
             ph("attend", lambda: tq.tq_attend(qv, logits, groups, G, vcache, kpg, scale, out=att, workspace=wsa,
                                               stream=stream))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        device_errors(tq, q, qv)
         pm = ph.mean_ms()
         sb = q.code_bytes + q.sign_bytes + 8 + 4 * G
         ab = 4 * G + qv.code_bytes + 8
@@ -967,6 +974,7 @@ def run_config(name, args, torch, tq, dev, stream, peak):
             ph("encode", lambda: tq.tq_encode(q, x, out=enc, workspace=wse, stream=stream))
             ph("topk", lambda: tq.tq_topk(q, y, enc, 10, workspace=ws, out=(vals, idx), stream=stream))
         ms = timed_steps(torch, dev, stream, step, steps, max(3, args.warmup), ph)
+        device_errors(tq, q)
         pm = ph.mean_ms()
         enc_flops = 2.0 * n * d * (d + d)
         topk_flops = 2.0 * nq * n * (d + d)

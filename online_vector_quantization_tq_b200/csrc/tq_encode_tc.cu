@@ -624,9 +624,6 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   const int pc = tid >> 7;  // column group (compute threads)
   const uint32_t lane = (uint32_t)(row & ~31) << 16;
 
-  // The next kernel may start in this one's tail: every kernel launched that
-  // way waits for this one before it touches memory.
-  sm100::pdl_launch_dependents();
   if (tid == 0) {
     for (int i = 0; i < 5; ++i) sm100::mbar_init(&bars[i], 1);
     sm100::fence_barrier_init();
@@ -649,10 +646,6 @@ k_encode_tc2(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *sTmem;
-  // The set-up above reads only the quantizer's tables and may overlap the
-  // previous kernel of the stream; x and the outputs are touched only once
-  // that kernel is complete.
-  sm100::pdl_wait();
 
   // Symmetric codebook (scaled 2^10): magnitude thresholds T_k, k = 1..HALF-1,
   // and centroid magnitudes C_k.  Each threshold test is the exact step
@@ -1029,9 +1022,6 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   const int pc = tid >> 7;
   const uint32_t lane = (uint32_t)(row & ~31) << 16;
 
-  // The next kernel may start in this one's tail: every kernel launched that
-  // way waits for this one before it touches memory.
-  sm100::pdl_launch_dependents();
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) sm100::mbar_init(&bars[i], 1);
     sm100::fence_barrier_init();
@@ -1049,10 +1039,6 @@ k_encode_tcg(const __grid_constant__ CUtensorMap xmap, const EncTCParams p) {
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *sTmem;
-  // The set-up above reads only the quantizer's tables and may overlap the
-  // previous kernel of the stream; x, the channel map and the outputs are
-  // touched only once that kernel is complete.
-  sm100::pdl_wait();
 
   constexpr float kBig = 1099511627776.0f;  // 2^40: exact steps sat(2^40 (|u| - T_k))
   float nTB[HALF], ndC[HALF];
@@ -1384,9 +1370,8 @@ tq_status launch_tcg(const void *x, int64_t n, int64_t ldx, const EncTCParams &p
     return TQ_ERR_CUDA;
   if (D == 32 && cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return TQ_ERR_CUDA;
-  // may start in the previous kernel's tail (set-up only until pdl_wait)
-  PdlLaunch L((unsigned)std::min(pp.ntiles, sms * per_sm), 128 * (D / 32) + 32, smem, st);
-  return cudaLaunchKernelEx(&L.cfg, kern, map, pp) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  kern<<<std::min(pp.ntiles, sms * per_sm), 128 * (D / 32) + 32, smem, st>>>(map, pp);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
 template <int D, int RP>
@@ -1466,9 +1451,8 @@ tq_status launch_tc2(const void *x, int64_t n, int64_t ldx, const EncTCParams &p
   auto kern = k_encode_tc2<D, W, QJL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TQ_ERR_CUDA;
-  // may start in the previous kernel's tail (set-up only until pdl_wait)
-  PdlLaunch L((unsigned)std::min(pp.ntiles, sms), 128 * (D / 32) + 32, smem, st);
-  return cudaLaunchKernelEx(&L.cfg, kern, map, pp) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  kern<<<std::min(pp.ntiles, sms), 128 * (D / 32) + 32, smem, st>>>(map, pp);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 }  // namespace
 

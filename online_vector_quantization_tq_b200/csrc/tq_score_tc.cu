@@ -47,10 +47,6 @@ struct ScoreTCParams {
   int64_t ldo;
   int accumulate;
   int nstages;  // key-row stages in the ring (bulk copies)
-  // nonzero: the kernel before this one in the stream is the query-side
-  // kernel, so the keys were complete before it let this kernel start and
-  // may be read before the dependency wait
-  int keys_ready;
   int *err;
 };
 
@@ -66,11 +62,7 @@ k_query_operand(const float *ytil, const float *p, int d, int m, int w, int64_t 
   // byte k of operand row n sits where the 128-byte-swizzled K-major tile
   // (three 128-byte K atoms of N rows) keeps it in shared memory
   auto at = [N](int n, int k) { return (k / 128) * (N * 128) + sm100::sw128_offset(n, (k % 128) / 16) + k % 16; };
-  // The previous kernel of the stream is complete from here on (this kernel
-  // may have started in its tail); only then may the scorer start, and it
-  // waits for this kernel where it reads qop and qsc.
-  sm100::pdl_wait();
-  sm100::pdl_launch_dependents();
+  sm100::pdl_launch_dependents();  // the scorer waits for this kernel only where it reads qop and qsc
   const int64_t qrow = blockIdx.x;
   const int64_t g = qrow / G, ql = qrow % G;
   const float *yr = ytil + qrow * d;
@@ -143,11 +135,7 @@ k_prep_operand(KernelTables kt, RowSource src, int64_t G, int N, int cexp, int8_
   __shared__ __align__(16) int8_t stg[kColsPerQuery][kScoreKBytes];
   const int64_t row = blockIdx.x;
   const int j = threadIdx.x;
-  // The previous kernel of the stream is complete from here on (this kernel
-  // may have started in its tail); only then may the scorer start, and it
-  // waits for this kernel where it reads qop and qsc.
-  sm100::pdl_wait();
-  sm100::pdl_launch_dependents();
+  sm100::pdl_launch_dependents();  // the scorer waits for this kernel only where it reads qop and qsc
   for (int i = j; i < kColsPerQuery * kScoreKBytes / 16; i += D) reinterpret_cast<uint4 *>(&stg[0][0])[i] = make_uint4(0, 0, 0, 0);
   float x = src.at(row, j);
 #pragma unroll
@@ -365,9 +353,6 @@ k_score_tc(const ScoreTCParams p) {
   volatile int *sAbort = reinterpret_cast<volatile int *>(sTmem + 1);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  // the next kernel may start in this one's tail: every kernel launched that
-  // way waits for this one before it touches memory
-  sm100::pdl_launch_dependents();
   const ScoreTmem tp(p.N, p.G);
   const int64_t t0 = (p.ntiles * blockIdx.x) / gridDim.x;
   const int64_t t1 = (p.ntiles * (blockIdx.x + 1)) / gridDim.x;
@@ -423,7 +408,6 @@ k_score_tc(const ScoreTCParams p) {
       tch[k] = p.tch[k];
       tcl[k] = p.tcl[k];
     }
-    if (!BULK && !p.keys_ready) sm100::pdl_wait();  // they read the keys themselves
     TileWalk tw(t0 + e, tpg);
     for (int it = e; it < n_it; it += kExpGroups, tw.advance(kExpGroups)) {
       const int64_t g = tw.g, kin = tw.tin * 128 + row;
@@ -632,10 +616,9 @@ k_score_tc(const ScoreTCParams p) {
       sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
       if (sb) sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
     };
-    // After the query-side kernel, the key stages that fit in the ring go
-    // first: the keys were complete before it let this kernel start; the
-    // query operands come from that kernel, which may still be running.
-    if (!p.keys_ready) sm100::pdl_wait();
+    // The key stages that fit in the ring go first: the keys were written
+    // before the query preparation started, so they need no wait; the query
+    // operands come from that kernel, which may still be running.
     if constexpr (BULK) {
       TileWalk tp(t0, tpg);
       for (; pre < n_it && pre < NS; ++pre, tp.advance(1)) issue_keys((int)pre, tp);
@@ -715,11 +698,9 @@ tq_status tc_score_queries(const tq_quantizer *q, const float *ytil, const float
   const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   const int64_t nq = groups * G;
   if (cudaMemsetAsync(qop, 0, tc_score_qop_bytes(q, groups, G), st) != cudaSuccess) return TQ_ERR_CUDA;
-  PdlLaunch L((unsigned)nq, 128, 0, st);
-  return cudaLaunchKernelEx(&L.cfg, k_query_operand, ytil, pq, q->d, q->m, q->w, G, N, q->score_cexp,
-                            q->kt.qjl_scale, qop, qsc) == cudaSuccess
-             ? TQ_OK
-             : TQ_ERR_CUDA;
+  k_query_operand<<<(unsigned)nq, 128, 0, st>>>(ytil, pq, q->d, q->m, q->w, G, N, q->score_cexp, q->kt.qjl_scale,
+                                                qop, qsc);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
 tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
@@ -729,7 +710,7 @@ tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, in
   const tq_status r = tc_score_queries(q, ytil, pq, groups, G, qop, qsc, st);
   if (r != TQ_OK) return r;
   return tc_score_keys(q, groups, G, kpg, key_base, nkeys, codes, signs, norms, out, ldo, accumulate, qop, qsc,
-                       true, st);
+                       st);
 }
 
 bool tc_score_y_supported(const tq_quantizer *q, int64_t G) {
@@ -741,26 +722,13 @@ tq_status tc_score_y_queries(const tq_quantizer *q, const RowSource &src, int64_
                              float4 *qsc, cudaStream_t st) {
   const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   const unsigned nq = (unsigned)(groups * G);
-  cudaError_t e;
   switch (q->d) {
-    case 32: {
-      PdlLaunch L(nq, 32, 0, st);
-      e = cudaLaunchKernelEx(&L.cfg, k_prep_operand<32>, q->kt, src, G, N, q->score_cexp, qop, qsc);
-      break;
-    }
-    case 64: {
-      PdlLaunch L(nq, 64, 0, st);
-      e = cudaLaunchKernelEx(&L.cfg, k_prep_operand<64>, q->kt, src, G, N, q->score_cexp, qop, qsc);
-      break;
-    }
-    case 128: {
-      PdlLaunch L(nq, 128, 0, st);
-      e = cudaLaunchKernelEx(&L.cfg, k_prep_operand<128>, q->kt, src, G, N, q->score_cexp, qop, qsc);
-      break;
-    }
+    case 32: k_prep_operand<32><<<nq, 32, 0, st>>>(q->kt, src, G, N, q->score_cexp, qop, qsc); break;
+    case 64: k_prep_operand<64><<<nq, 64, 0, st>>>(q->kt, src, G, N, q->score_cexp, qop, qsc); break;
+    case 128: k_prep_operand<128><<<nq, 128, 0, st>>>(q->kt, src, G, N, q->score_cexp, qop, qsc); break;
     default: return TQ_ERR_UNSUPPORTED;
   }
-  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
 tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups, int64_t G, int64_t kpg,
@@ -768,13 +736,12 @@ tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups
                      int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st) {
   const tq_status r = tc_score_y_queries(q, src, groups, G, qop, qsc, st);
   if (r != TQ_OK) return r;
-  return tc_score_keys(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, ldo, accumulate, qop, qsc, true, st);
+  return tc_score_keys(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, ldo, accumulate, qop, qsc, st);
 }
 
 tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
                         int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
-                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, bool keys_ready,
-                        cudaStream_t st) {
+                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, cudaStream_t st) {
   const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   ScoreTCParams prm{};
   prm.d = q->d;
@@ -803,7 +770,6 @@ tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_
   prm.out = out;
   prm.ldo = ldo;
   prm.accumulate = accumulate;
-  prm.keys_ready = keys_ready ? 1 : 0;
   prm.err = q->d_err;
   const int ng = q->d / 32, cwords = q->w * ng;
   const size_t stage_bytes = ((size_t)128 * (cwords + ng) * 4 + 1023) / 1024 * 1024;
@@ -831,13 +797,20 @@ tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = std::min<int64_t>(prm.ntiles, (int64_t)sms);
   if (grid <= 0) return TQ_OK;
-  // Programmatic dependent launch: the scorer may start in the previous
-  // kernel's tail.  After the query-side kernel (keys_ready) it sets up and
-  // loads keys while that kernel still runs; otherwise its threads wait for
-  // the previous kernel before they read keys.  Query operands and scales are
-  // read only after the wait.
-  PdlLaunch L((unsigned)grid, kScoreThreads, smem, st);
-  cudaLaunchConfig_t &cfg = L.cfg;
+  // Programmatic dependent launch: after the query-side kernel (which lets
+  // its dependents start at once) the scorer sets up and loads keys while
+  // that kernel still runs; its threads wait for it where they read qop and
+  // qsc.  After any other kernel it starts as usual.
+  cudaLaunchAttribute pdl{};
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kScoreThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
 #define TQ_SC(WW, NGG)                                                                                   \
   {                                                                                                      \
     auto kern = bulk ? k_score_tc<WW, NGG, true> : k_score_tc<WW, NGG, false>;                           \

@@ -113,9 +113,11 @@ __device__ __forceinline__ void fence_proxy_async() {
 // programmatic stream serialization, start before it has finished; the
 // dependent kernel's threads call pdl_wait before they read anything the
 // first kernel writes (it returns once that kernel has completed and its
-// writes are visible).  Without the launch attribute, or after a kernel that
-// never calls pdl_launch_dependents, the dependent kernel starts after the
-// previous one as usual and pdl_wait returns at once.
+// writes are visible), and before they allocate TMEM: an allocation that
+// waits for another kernel's columns also holds up that kernel's MMAs on the
+// SM.  Without the launch attribute, or after a kernel that never calls
+// pdl_launch_dependents, the dependent kernel starts after the previous one
+// as usual and pdl_wait returns at once.
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -420,27 +422,4 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 }  // namespace sm100
-}  // namespace tq
-
-namespace tq {
-// Host: launch configuration with programmatic stream serialization.  The
-// kernel may start while the previous kernel of its stream is still running,
-// once that kernel calls pdl_launch_dependents (every CTA) or finishes; the
-// kernel calls pdl_wait before it touches memory the previous one may write.
-struct PdlLaunch {
-  cudaLaunchAttribute attr;
-  cudaLaunchConfig_t cfg;
-  PdlLaunch(unsigned grid, unsigned block, size_t smem, cudaStream_t st) : attr{}, cfg{} {
-    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr.val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-  }
-  PdlLaunch(const PdlLaunch &) = delete;  // cfg points at attr
-  PdlLaunch &operator=(const PdlLaunch &) = delete;
-};
 }  // namespace tq
