@@ -716,3 +716,50 @@ def test_score_in_two_halves(tq, d, b, rot, G, mse):
             r = {k: v[keys] for k, v in rep.ref.items()}
             check_scores(s[rows], o.score(yt[0][rows], yt[1][rows], r, t), r["norm"],
                          np.linalg.norm(y[rows], axis=1), d, rep.skip_rows[keys])
+
+
+def test_back_to_back_steps(tq):
+    """Steps of the split-precision KV layer (two gathered encodes, then two
+    scorers, the second accumulating) queued back to back with no host
+    synchronisation in between: no kernel records a failed wait, and the last
+    step's logits equal those of the same calls run one at a time.  Then the
+    scorer right after the encode that wrote its keys (tq_score_prepared on
+    the same stream, no synchronisation) against the synchronised result."""
+    n, groups, G = 32768, 8, 4
+    xs = np.stack([wl.kv_head_keys(h, n) for h in range(groups)])
+    x_dev = dev(xs.reshape(-1, 128), torch.bfloat16)
+    y_dev = dev(wl.kv_queries())
+    sel, rest = tq.tq_outlier_channels(x_dev, groups, n, 32)
+    (da, ba), (db, bb) = wl.MIXED_SPLIT
+    qa, qb = tq.tq_codebook(da, ba, seed=0), tq.tq_codebook(db, bb, seed=0)
+    encs = [(qa.empty_encoded(groups * n), qb.empty_encoded(groups * n)) for _ in range(2)]
+    out = torch.empty((groups * G, n), device="cuda")
+
+    def step(i):
+        (ea, eb), (ra, rb) = encs[i % 2], encs[(i + 1) % 2]
+        tq.tq_encode(qa, x_dev, out=ea, chan=sel, chan_rows=n)
+        tq.tq_encode(qb, x_dev, out=eb, chan=rest, chan_rows=n)
+        tq.tq_score(qa, y_dev, groups, G, ra, n, out=out, ychan=sel)
+        tq.tq_score(qb, y_dev, groups, G, rb, n, out=out, accumulate=True, ychan=rest)
+
+    for i in range(6):
+        step(i)
+    tq.tq_sync_check(qa)
+    tq.tq_sync_check(qb)
+    got = out.clone()
+    ra, rb = encs[(5 + 1) % 2]
+    ref = tq.tq_score(qa, y_dev, groups, G, ra, n, ychan=sel)
+    torch.cuda.synchronize()
+    tq.tq_score(qb, y_dev, groups, G, rb, n, out=ref, accumulate=True, ychan=rest)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+
+    q = tq.tq_codebook(128, 4, seed=0)
+    ws = tq.tq_score_prepare(q, y_dev, groups, G)
+    enc = q.empty_encoded(groups * n)
+    enc.codes.zero_()
+    tq.tq_encode(q, x_dev, out=enc)
+    got = tq.tq_score_prepared(q, groups, G, enc, n, ws)
+    tq.tq_sync_check(q)
+    torch.cuda.synchronize()
+    assert torch.equal(got, tq.tq_score(q, y_dev, groups, G, enc, n))
