@@ -58,7 +58,7 @@ CSRC = os.path.join(ROOT, "online_vector_quantization_tq_b200", "csrc")
 TRAFFIC = {
     # kernel@workload: (source file, digest, bytes per launch, the capture)
     "k_encode_tc2@kv": ("tq_encode_tc.cu", "ba567bfd970bd1b8", 326984192, "kv workload, launch 4, ncu --set full"),
-    "k_score_tc@kv": ("tq_score_tc.cu", "ad79fc3f164546d5", 79580416, "kv workload, launch 4, ncu --set full"),
+    "k_score_tc@kv": ("tq_score_tc.cu", "5afa1e3f15b38586", 79768320, "kv workload, launch 4, ncu --set full"),
     "k_attend_split@decode_attend": ("tq_attend.cu", "ba7f8d0459655239", 615365632, "decode_attend workload, launch 3, ncu --set full"),
 }
 

@@ -294,9 +294,11 @@ tq_status tq_score_prepared(const tq_quantizer *q, int64_t groups, int64_t G, co
   switch (path) {
     case kPathTcY:
     case kPathTc:
+      // the kernel before this call may be anything (an encode of these keys):
+      // the scorer waits for it before reading keys or allocating TMEM
       return tc_score_keys(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, kpg, accumulate,
                            reinterpret_cast<const int8_t *>(ws + L.qop), reinterpret_cast<const float4 *>(ws + L.qsc),
-                           s);
+                           false, s);
     case kPathDense:
       // the dense path's own scratch follows the prepared queries in the workspace
       return dense_score(q, ytil, p, nq, G, kpg, 0, kpg, codes, signs, norms, out, kpg, accumulate, ws + L.dense,

@@ -108,10 +108,13 @@ size_t tc_score_qop_bytes(const tq_quantizer *q, int64_t groups, int64_t G);
 // the query half from prepared queries (y~, p)
 tq_status tc_score_queries(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
                            int8_t *qop, float4 *qsc, cudaStream_t st);
-// the key half: keys [key_base, key_base + nkeys) of every group
+// the key half: keys [key_base, key_base + nkeys) of every group.  keys_ready:
+// the previous kernel of the stream is the query half (the scorer may read
+// keys and allocate TMEM before its dependency wait); otherwise it waits first
 tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
                         int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
-                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, cudaStream_t st);
+                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, bool keys_ready,
+                        cudaStream_t st);
 tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, int64_t groups, int64_t G,
                    int64_t kpg, int64_t key_base, int64_t nkeys, const void *codes, const void *signs,
                    const float *norms, float *out, int64_t ldo, int accumulate, int8_t *qop, float4 *qsc,

@@ -47,6 +47,11 @@ struct ScoreTCParams {
   int64_t ldo;
   int accumulate;
   int nstages;  // key-row stages in the ring (bulk copies)
+  // nonzero: the kernel before this one in the stream is the query-side
+  // kernel (launched normally, so the keys were complete before it started,
+  // and it uses no TMEM): keys may be read, and TMEM allocated, before the
+  // dependency wait
+  int keys_ready;
   int *err;
 };
 
@@ -381,6 +386,10 @@ k_score_tc(const ScoreTCParams p) {
     *sAbort = 0;
     sm100::fence_barrier_init();
   }
+  // After any other kernel, wait for it first: it may have written the keys,
+  // and a TMEM allocation that has to wait for another kernel's columns also
+  // holds up that kernel's MMAs on this SM.
+  if (!p.keys_ready) sm100::pdl_wait();
   if (warp == kMmaWarp) {
     sm100::tmem_alloc(sTmem, (uint32_t)tp.ncols);
     sm100::tmem_relinquish();
@@ -616,9 +625,10 @@ k_score_tc(const ScoreTCParams p) {
       sm100::bulk_load(st, p.codes + key0 * CW, cb, &bars[SM::kFull + slot]);
       if (sb) sm100::bulk_load(st + SM::kCodeBytes, p.signs + key0 * NG, sb, &bars[SM::kFull + slot]);
     };
-    // The key stages that fit in the ring go first: the keys were written
-    // before the query preparation started, so they need no wait; the query
-    // operands come from that kernel, which may still be running.
+    // The key stages that fit in the ring go first: after the query-side
+    // kernel (keys_ready) the keys were complete before it started, and
+    // otherwise this thread has waited already; the query operands come from
+    // that kernel, which may still be running.
     if constexpr (BULK) {
       TileWalk tp(t0, tpg);
       for (; pre < n_it && pre < NS; ++pre, tp.advance(1)) issue_keys((int)pre, tp);
@@ -710,7 +720,7 @@ tq_status tc_score(const tq_quantizer *q, const float *ytil, const float *pq, in
   const tq_status r = tc_score_queries(q, ytil, pq, groups, G, qop, qsc, st);
   if (r != TQ_OK) return r;
   return tc_score_keys(q, groups, G, kpg, key_base, nkeys, codes, signs, norms, out, ldo, accumulate, qop, qsc,
-                       st);
+                       true, st);
 }
 
 bool tc_score_y_supported(const tq_quantizer *q, int64_t G) {
@@ -736,12 +746,13 @@ tq_status tc_score_y(const tq_quantizer *q, const RowSource &src, int64_t groups
                      int accumulate, int8_t *qop, float4 *qsc, cudaStream_t st) {
   const tq_status r = tc_score_y_queries(q, src, groups, G, qop, qsc, st);
   if (r != TQ_OK) return r;
-  return tc_score_keys(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, ldo, accumulate, qop, qsc, st);
+  return tc_score_keys(q, groups, G, kpg, 0, kpg, codes, signs, norms, out, ldo, accumulate, qop, qsc, true, st);
 }
 
 tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_t kpg, int64_t key_base,
                         int64_t nkeys, const void *codes, const void *signs, const float *norms, float *out,
-                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, cudaStream_t st) {
+                        int64_t ldo, int accumulate, const int8_t *qop, const float4 *qsc, bool keys_ready,
+                        cudaStream_t st) {
   const int N = (int)((kColsPerQuery * G + 15) / 16 * 16);
   ScoreTCParams prm{};
   prm.d = q->d;
@@ -770,6 +781,7 @@ tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_
   prm.out = out;
   prm.ldo = ldo;
   prm.accumulate = accumulate;
+  prm.keys_ready = keys_ready ? 1 : 0;
   prm.err = q->d_err;
   const int ng = q->d / 32, cwords = q->w * ng;
   const size_t stage_bytes = ((size_t)128 * (cwords + ng) * 4 + 1023) / 1024 * 1024;
@@ -800,7 +812,8 @@ tq_status tc_score_keys(const tq_quantizer *q, int64_t groups, int64_t G, int64_
   // Programmatic dependent launch: after the query-side kernel (which lets
   // its dependents start at once) the scorer sets up and loads keys while
   // that kernel still runs; its threads wait for it where they read qop and
-  // qsc.  After any other kernel it starts as usual.
+  // qsc.  After any other kernel it waits for that kernel before anything
+  // else (keys_ready = 0).
   cudaLaunchAttribute pdl{};
   pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl.val.programmaticStreamSerializationAllowed = 1;
