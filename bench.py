@@ -57,9 +57,9 @@ CSRC = os.path.join(ROOT, "online_vector_quantization_tq_b200", "csrc")
 # those sources are unchanged; otherwise the roofline's traffic is null.
 TRAFFIC = {
     # kernel@workload: (source file, digest, bytes per launch, the capture)
-    "k_encode_tc2@kv": ("tq_encode_tc.cu", "ba567bfd970bd1b8", 326984192, "kv workload, launch 4, ncu --set full"),
+    "k_encode_tc2@kv": ("tq_encode_tc.cu", "9831e14a2c4ee1a7", 326491392, "kv workload, launch 4, ncu --set full"),
     "k_score_tc@kv": ("tq_score_tc.cu", "5afa1e3f15b38586", 79768320, "kv workload, launch 4, ncu --set full"),
-    "k_attend_split@decode_attend": ("tq_attend.cu", "ba7f8d0459655239", 615365632, "decode_attend workload, launch 3, ncu --set full"),
+    "k_attend_split@decode_attend": ("tq_attend.cu", "8a7739e9493e3030", 616206848, "decode_attend workload, launch 3, ncu --set full"),
 }
 
 
