@@ -62,3 +62,41 @@ def test_traffic_is_null_once_the_source_changes(monkeypatch):
     assert b.traffic_for("k") == (None, None)
     assert b.traffic_for("old", "w") == (None, None)
     assert b.traffic_for("missing", "w") == (None, None)
+
+
+def test_device_errors_checks_every_quantizer():
+    """After a timed region the bench asks the library for each quantizer's
+    error word; an error (a kernel that gave up a bounded wait) fails the run."""
+    b = _bench()
+    seen = []
+
+    class FakeTq:
+        @staticmethod
+        def tq_sync_check(q):
+            seen.append(q)
+            if q == "bad":
+                raise RuntimeError("a kernel gave up a bounded wait")
+
+    b.device_errors(FakeTq, "qa", "qb")
+    assert seen == ["qa", "qb"]
+    import pytest
+    with pytest.raises(RuntimeError):
+        b.device_errors(FakeTq, "qa", "bad", "qc")
+
+
+def test_phases_off_run_the_work_without_events():
+    """Timed steps run with the phase recorder switched off: the work still
+    runs, and no CUDA event is created (so none sits between two kernels)."""
+    b = _bench()
+
+    class NoCuda:
+        class cuda:
+            @staticmethod
+            def Event(**kw):
+                raise AssertionError("no event while phases are off")
+
+    ph = b.Phases(NoCuda, None)
+    ph.enabled = False
+    ran = []
+    ph("encode", lambda: ran.append(1))
+    assert ran == [1] and ph.ev == {}
