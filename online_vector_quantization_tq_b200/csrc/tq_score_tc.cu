@@ -418,6 +418,10 @@ k_score_tc(const ScoreTCParams p) {
       tcl[k] = p.tcl[k];
     }
     TileWalk tw(t0 + e, tpg);
+    // ring slot of tile it and the parity of its fill, kept as counters
+    // (it % NS and (it / NS) & 1 without a division per tile)
+    int slot = e % NS;
+    uint32_t fill_ph = (uint32_t)((e / NS) & 1);
     for (int it = e; it < n_it; it += kExpGroups, tw.advance(kExpGroups)) {
       const int64_t g = tw.g, kin = tw.tin * 128 + row;
       const bool valid = kin < p.nkeys;
@@ -427,8 +431,7 @@ k_score_tc(const ScoreTCParams p) {
 #pragma unroll
       for (int k = 0; k < NG; ++k) sw[k] = 0u;
       if constexpr (BULK) {
-        const int slot = it % NS;
-        if (!__all_sync(0xffffffffu, wait(SM::kFull + slot, (uint32_t)((it / NS) & 1), 21))) break;
+        if (!__all_sync(0xffffffffu, wait(SM::kFull + slot, fill_ph, 21))) break;
         const uint8_t *st = sStage + slot * SM::kStageBytes;
         if (valid) {
           if constexpr (CW % 4 == 0) {
@@ -454,6 +457,7 @@ k_score_tc(const ScoreTCParams p) {
         }
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(&bars[SM::kEmpty + slot]);
+        for (slot += kExpGroups; slot >= NS; slot -= NS) fill_ph ^= 1u;
       } else {
         if (valid) {
           const int64_t key = g * p.kpg + p.key_base + kin;
