@@ -58,7 +58,7 @@ CSRC = os.path.join(ROOT, "online_vector_quantization_tq_b200", "csrc")
 TRAFFIC = {
     # kernel@workload: (source file, digest, bytes per launch, the capture)
     "k_encode_tc2@kv": ("tq_encode_tc.cu", "9831e14a2c4ee1a7", 326491392, "kv workload, launch 4, ncu --set full"),
-    "k_score_tc@kv": ("tq_score_tc.cu", "5afa1e3f15b38586", 79768320, "kv workload, launch 4, ncu --set full"),
+    "k_score_tc@kv": ("tq_score_tc.cu", "29c8a83c49dff57f", 79304448, "kv workload, launch 4, ncu --set full"),
     "k_attend_split@decode_attend": ("tq_attend.cu", "8a7739e9493e3030", 616206848, "decode_attend workload, launch 3, ncu --set full"),
 }
 
